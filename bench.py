@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""SinkRouter decode-attention benchmark on B200.
+
+One step = one routed decode step of one attention layer (sr_route then
+sr_decode_attention, through the C ABI) on synthetic inputs shaped like the
+Llama-3.1-8B 128K-context decode layer: batch 1, 32 query / 8 KV heads,
+head_dim 128, bf16 cache, 4 of 8 KV groups planted sinks, tau 0.6.
+
+Prints one JSON line (rank 0): µs per layer-step (lower is better), effective
+HBM GB/s over the bytes the step must move, the roofline of the decode kernel
+against the measured HBM copy bandwidth, the same kernel with routing disabled
+(tau = +inf), the fp64 CPU oracle on this host's cores, an end-to-end figure
+with host buffers, and the SM clocks seen during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own independent layer-step (the
+units of a decode step share nothing); time is the max over ranks and the value
+is that time divided by all layer-steps of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention µs/layer-step and effective HBM GB/s (% of peak) at 128K/512K ctx"
+UNIT = "us/layer-step"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_128k.md")
+DECODE_SOURCE = os.path.join(ROOT, "kv_cache_routing_sr_b200", "csrc", "sr_decode.cu")
+L2_FLUSH_BYTES = 256 << 20
+
+NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="llama8b_128k")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 512K sink-fraction sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+# ---------------------------------------------------------------------------------------
+# helpers shared by both arms
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            v = json.load(f).get("hbm_gbs")
+        if v:
+            return float(v), "measured"
+    except (OSError, ValueError):
+        pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """dram bytes per launch of the decode kernel from the committed ncu summary,
+    valid only while the kernel source still has the hash it was captured at."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+        src = hashlib.sha256(open(DECODE_SOURCE, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^decode_source_sha256:\s*([0-9a-f]+)", text, re.M)
+    if not m_t or not m_h or m_h.group(1) != src:
+        return None
+    return float(m_t.group(1))
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def active_units_of(active_list_cpu):
+    n = int(active_list_cpu[0])
+    return [int(u) for u in active_list_cpu[1:1 + n]]
+
+
+def describe_config(x, n_active, n_gpus):
+    return {
+        "workload": x.workload.name,
+        "description": x.workload.description,
+        "batch": x.batch, "context": x.max_seq_len, "q_heads": x.n_q_heads, "kv_heads": x.n_kv_heads,
+        "head_dim": 128, "tau": x.tau, "units": x.batch * x.n_kv_heads, "active_units": n_active,
+        "seq_lens": [int(v) for v in x.seq_lens.cpu().tolist()][:8],
+        "l2": "inputs (K/V caches) larger than L2, and a 256 MiB L2 flush write between steps, outside the "
+              "per-step events",
+        "parallelism": f"replicas x{n_gpus} (independent layer-steps, no collective on the data path)",
+    }
+
+
+# ---------------------------------------------------------------------------------------
+# clock sampling (NVML reads only)
+
+class ClockSampler:
+    def __init__(self, torch_device_index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device_index)
+            h = None
+            try:
+                bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return int(fn(self.h))
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                self.samples.append((mhz, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if not self.ok:
+            return
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        self._stop.set()
+        self._t.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [name for b, name in NVML_REASONS.items() if bits & b]
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+
+def time_steps(native, dec, x, tau, steps, flush, dist, barrier):
+    """Run `steps` layer-steps; returns per-step (total, route, decode) ms lists
+    measured with CUDA events on the current stream."""
+    import torch
+    st = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)  # evict the previous step's lines from L2
+        ev[i][0].record(st)
+        native.route(x.q, x.k0, tau, dec.route_mask, dec.active_list)
+        ev[i][1].record(st)
+        native.decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, dec.active_list, dec.out,
+                                0, dec.workspace)
+        ev[i][2].record(st)
+    torch.cuda.synchronize()
+    barrier()
+    tot = [e[0].elapsed_time(e[2]) for e in ev]
+    rte = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    return tot, rte, dec_ms
+
+
+def measure_workload(native, inputs, x, steps, warmup, flush, dist, barrier, peak):
+    """Routed and routing-disabled timings of one workload on this GPU."""
+    import torch
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
+    for _ in range(warmup):
+        dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+    torch.cuda.synchronize()
+    err = dec.workspace.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err} after warm-up")
+    act = active_units_of(dec.active_list.cpu())
+    sl = x.seq_lens.cpu().tolist()
+    need = inputs.needed_bytes(sl, act, x.n_kv_heads, x.n_q_heads, x.batch)
+    need_all = inputs.needed_bytes(sl, range(x.batch * x.n_kv_heads), x.n_kv_heads, x.n_q_heads, x.batch)
+    tot, rte, dms = time_steps(native, dec, x, x.tau, steps, flush, dist, barrier)
+    for _ in range(warmup):
+        dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, float("inf"))
+    tot_d, _, dms_d = time_steps(native, dec, x, float("inf"), steps, flush, dist, barrier)
+    return dict(dec=dec, active=act, need=need, need_all=need_all, tot=tot, route=rte, decode=dms,
+                tot_disabled=tot_d, decode_disabled=dms_d)
+
+
+def e2e_measure(native, x, steps):
+    """Same step through the public API with host buffers: pinned host -> device
+    copies of every input, the two calls, and device -> host of the outputs,
+    all inside the timed region."""
+    import torch
+    names = ["q", "k_cache", "v_cache", "k0", "v0", "seq_lens"]
+    host = {n: getattr(x, n).cpu().pin_memory() for n in names}
+    dev = {n: torch.empty_like(getattr(x, n)) for n in names}
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
+    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    mask_h = torch.empty(dec.route_mask.shape, dtype=dec.route_mask.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + mask_h.numel()
+    st = torch.cuda.current_stream()
+
+    def one():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        dec.step(dev["q"], dev["k_cache"], dev["v_cache"], dev["k0"], dev["v0"], dev["seq_lens"], x.tau)
+        out_h.copy_(dec.out, non_blocking=True)
+        mask_h.copy_(dec.route_mask, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del dev, host
+    return ms, h2d, d2h
+
+
+def oracle_layer_step_us(x_cpu, budget_s, min_reps=1):
+    """The fp64 oracle, as it stands, on whole layer-steps of this workload."""
+    import torch
+
+    import oracle
+    tau = float(torch.tensor(x_cpu.tau, dtype=torch.float32))
+    mask, active, _ = oracle.route(x_cpu.q, x_cpu.k0, tau)
+    n_act = int(active[0])
+    threads = max(1, min(os.cpu_count() or 1, max(1, n_act)))
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.routed_attention(x_cpu.q, x_cpu.k_cache, x_cpu.v_cache, x_cpu.k0, x_cpu.v0, x_cpu.seq_lens, tau,
+                                n_threads=threads)
+        reps += 1
+        if reps >= min_reps and time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return el / reps * 1e6, threads, reps, el
+
+
+def run_ours(args):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from kv_cache_routing_sr_b200 import inputs, native
+
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.gpus > 1 and world == 1:
+        raise SystemExit("--gpus > 1 needs torchrun (one process per GPU)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peak, peak_kind = hbm_peak()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    x = inputs.make(args.config, seed=args.seed + 1000 * rank, device=dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_wall = time.perf_counter()
+    r = measure_workload(native, inputs, x, args.steps, args.warmup, flush, dist, barrier, peak)
+    t_wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+
+    K = args.steps
+    sum_ms = max_over_ranks(sum(r["tot"]))
+    sum_ms_dis = max_over_ranks(sum(r["tot_disabled"]))
+    us_step = sum_ms * 1e3 / K  # slowest rank's µs per layer-step
+    value = sum_ms * 1e3 / (K * world)  # whole job: time / all layer-steps of all ranks
+    dec_us = statistics.mean(r["decode"]) * 1e3
+    route_us = statistics.median(r["route"]) * 1e3
+    eff_gbs = r["need"] / (us_step * 1e-6) / 1e9
+    us_dis = sum_ms_dis * 1e3 / K
+    eff_gbs_dis = r["need_all"] / (us_dis * 1e-6) / 1e9
+    achieved = r["need"] / (dec_us * 1e-6) / 1e9
+    traffic = profiled_traffic()
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(us_step / 1e3, 6), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
+        "config": describe_config(x, len(r["active"]), world),
+        "effective_gbs": round(eff_gbs, 1), "frac_of_hbm_peak": round(eff_gbs / peak, 4),
+        "route_us_median": round(route_us, 3), "decode_us_mean": round(dec_us, 3),
+        "step_us_p10_p50_p90": [round(statistics.quantiles(r["tot"], n=10)[i] * 1e3, 3) for i in (0, 4, 8)],
+        "needed_bytes_per_step": r["need"],
+        "routing_disabled": {"us_per_layer_step": round(us_dis, 3), "effective_gbs": round(eff_gbs_dis, 1),
+                             "frac_of_hbm_peak": round(eff_gbs_dis / peak, 4),
+                             "decode_us_mean": round(statistics.mean(r["decode_disabled"]) * 1e3, 3),
+                             "speedup_routed": round(us_dis / us_step, 3),
+                             "active_fraction": round(len(r["active"]) / (x.batch * x.n_kv_heads), 4)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "sinkrouter decode_kernel (persistent split-K scan + reduction)",
+                     "algorithmic_bytes_per_launch": r["need"], "peak_source": f"{peak_kind} HBM copy"},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+        "timed_wall_s": round(t_wall, 3),
+        "impl": "ours",
+    }
+    del r
+    if world == 1 and not args.no_sweep:
+        sweep = []
+        for frac in (0.0, 0.25, 0.5, 0.75, 1.0):
+            x5 = inputs.make("llama8b_512k", seed=args.seed, device=dev, sink_fraction=frac)
+            s5 = measure_workload(native, inputs, x5, max(20, min(K, 50)), args.warmup, flush, dist, barrier, peak)
+            u5 = statistics.mean(s5["tot"]) * 1e3
+            d5 = statistics.mean(s5["decode"]) * 1e3
+            ud5 = statistics.mean(s5["tot_disabled"]) * 1e3
+            sweep.append({"sink_fraction": frac, "us_per_layer_step": round(u5, 2),
+                          "effective_gbs": round(s5["need"] / (u5 * 1e-6) / 1e9, 1),
+                          "decode_kernel_gbs": round(s5["need"] / (d5 * 1e-6) / 1e9, 1),
+                          "decode_frac_of_peak": round(s5["need"] / (d5 * 1e-6) / 1e9 / peak, 4),
+                          "routing_disabled_us": round(ud5, 2), "speedup_routed": round(ud5 / u5, 3)})
+            del x5, s5
+            torch.cuda.empty_cache()
+        line["sweep_512k"] = sweep
+    if not args.no_e2e:
+        ms, h2d, d2h = e2e_measure(native, x, args.e2e_steps)
+        ms = max_over_ranks(ms)
+        line["e2e"] = {"value": round(ms * 1e3 / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                       "note": "pinned host buffers; every input (caches included) copied each step"}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        xc = x.to("cpu")
+        us, threads, reps, el = oracle_layer_step_us(xc, args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{reps} whole layer-steps of {x.workload.name} "
+                                          f"({x.batch * x.n_kv_heads} units) in {el:.1f} s, fp64 C oracle, "
+                                          f"{threads} threads (one per active unit, capped at the host cores)",
+                                "host_cores": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    from kv_cache_routing_sr_b200 import inputs
+    x = inputs.make(args.config, seed=args.seed, device="cpu")
+    tau = float(torch.tensor(x.tau, dtype=torch.float32))
+    import oracle
+    mask, active, _ = oracle.route(x.q, x.k0, tau)
+    n_act = int(active[0])
+    threads = max(1, min(os.cpu_count() or 1, max(1, n_act)))
+    # Each step is one whole layer-step unless that would make the run exceed
+    # about three minutes; then a step is a bounded sample of the active units,
+    # scaled to the whole layer-step.
+    t0 = time.perf_counter()
+    oracle.routed_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, tau, n_threads=threads)
+    one = time.perf_counter() - t0
+    total_steps = args.steps + args.warmup
+    units = None
+    scale = 1.0
+    sample = "whole layer-step"
+    if one * total_steps > 180.0 and n_act > 1:
+        keep = max(1, int(n_act * 180.0 / (one * total_steps)))
+        act = [int(u) for u in active[1:1 + n_act]]
+        units = act[:keep]
+        scale = n_act / keep
+        sample = f"{keep} of {n_act} active units per step, scaled by {scale:.2f}"
+    times = []
+    for i in range(total_steps):
+        t0 = time.perf_counter()
+        mask, _, _ = oracle.route(x.q, x.k0, tau)
+        oracle.decode(x.q, x.k_cache, x.v_cache, x.v0, x.seq_lens, mask, units=units, n_threads=threads)
+        el = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(el * scale)
+    us = statistics.mean(times) * 1e6
+    line = {
+        "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": describe_config(x, n_act, 1) | {"parallelism": "host cores (CPU oracle)"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample, "host_cores": os.cpu_count()},
+        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/*
+ * sinkrouter.h -- C ABI of libsinkrouter.so: SinkRouter single-token decode
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (SinkRouter README, github.com/streamer-AP/SinkRouter, the
+ * decode-time procedure list; sota2 summary of "SinkRouter: Sink-Aware Routing
+ * for Efficient Long-Context Decoding ...", Abstract): at each decode step, every
+ * GQA KV-head group is routed before the long KV-cache scan by comparing its
+ * RoPE'd query heads with the cached position-0 key. Sink groups skip the scan
+ * and return the position-0 value; active groups run split-K softmax attention
+ * over the whole cache with an in-kernel reduction across splits.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller, contiguous,
+ *    row-major, 16-byte aligned. The library never allocates or frees memory.
+ *  - bf16 tensors are IEEE bfloat16 bit patterns (2 bytes per element).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Calls are asynchronous on that stream and never synchronise the
+ *    host, except sr_get_device_error, which synchronises `stream`.
+ *  - Host-visible argument errors return a status and launch nothing. Errors
+ *    that depend on device data (seq_lens, active_list contents) cannot be seen
+ *    on the host: the kernels clamp or skip and set bits in a device error word
+ *    kept in the workspace (sr_get_device_error). No kernel traps.
+ *  - A "unit" is one (sequence b, KV head g) pair, flat index u = b*Hkv + g.
+ *    Query head h belongs to KV head g = h / M, M = Hq / Hkv (contiguous blocks).
+ */
+#ifndef SINKROUTER_H
+#define SINKROUTER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Shapes of one attention layer's decode step. */
+typedef struct sr_dims {
+    int32_t batch;       /* B >= 1 */
+    int32_t n_q_heads;   /* Hq, a multiple of n_kv_heads */
+    int32_t n_kv_heads;  /* Hkv >= 1; group size M = Hq / Hkv must be 1, 2, 4 or 8 */
+    int32_t head_dim;    /* d; must be 128 */
+    int32_t max_seq_len; /* Lmax >= 1: positions allocated per unit in the caches */
+} sr_dims;
+
+typedef enum sr_status {
+    SR_OK = 0,
+    SR_ERR_INVALID_ARG = 1, /* null or misaligned pointer, non-positive size, bad n_splits */
+    SR_ERR_UNSUPPORTED = 2, /* shape the kernels do not implement (d != 128, M not in {1,2,4,8},
+                               B*Hkv > SR_MAX_UNITS) */
+    SR_ERR_WORKSPACE = 3,   /* workspace pointer null/misaligned or smaller than needed */
+    SR_ERR_CUDA = 4         /* a CUDA runtime call or kernel launch failed */
+} sr_status;
+
+/* Largest B*Hkv the kernels accept. */
+#define SR_MAX_UNITS 16384
+/* Largest forced split count per unit. */
+#define SR_MAX_SPLITS 4096
+
+/* Bits of the device error word (sr_get_device_error). */
+#define SR_DEVERR_SEQ_LEN 1     /* a seq_lens entry was outside [1, Lmax]; it was clamped */
+#define SR_DEVERR_ACTIVE_LIST 2 /* active_list count or an entry was out of range or out of
+                                   order; the bad entries were skipped */
+#define SR_DEVERR_TIMEOUT 4     /* a pipeline wait exceeded its time bound (a bug, never
+                                   expected); outputs of that launch are invalid and the
+                                   workspace must be re-initialised with sr_workspace_init */
+
+/*
+ * sr_route -- cosine routing of every unit (README decode list: compare the RoPE
+ * query with the cached position-0 key and route each KV group before the scan;
+ * README routing controls: cosine threshold). For unit (b, g):
+ *     c_h = <q_h, k0_g> / (|q_h| |k0_g|)   for the M query heads h of group g
+ *           (c_h = 0 when either norm is 0)
+ *     s_g = min_h c_h;   sink  <=>  s_g >= tau
+ * The min over heads and the ">=" are this library's reading; the pages leave
+ * the combination open. Computed in fp32 from the bf16 inputs.
+ *
+ *   q           bf16 [B, Hq, d]   decode query after RoPE
+ *   k0          bf16 [B, Hkv, d]  cached position-0 key (RoPE at position 0 is
+ *                                 the identity)
+ *   tau         threshold; +INFINITY routes nothing, -INFINITY routes every unit
+ *   route_mask  out uint8 [B*Hkv]: 1 = sink, 0 = active
+ *   active_list out int32 [1 + B*Hkv]: [0] = number of active units n, then
+ *               their flat indices in ascending order; entries past 1+n are
+ *               left untouched
+ * One launch; no workspace. Errors: SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED,
+ * SR_ERR_CUDA.
+ */
+sr_status sr_route(const sr_dims *dims, const void *q, const void *k0, float tau,
+                   uint8_t *route_mask, int32_t *active_list, void *stream);
+
+/*
+ * sr_decode_workspace_bytes -- size of the workspace sr_decode_attention needs
+ * for any call with these dims and n_splits <= max_splits (0 = automatic
+ * splits only). Holds the device error word, one self-resetting arrival
+ * counter per unit and the fp32 split partials (m, l, O) of every split.
+ * Returns 0 for invalid or unsupported dims.
+ */
+size_t sr_decode_workspace_bytes(const sr_dims *dims, int32_t max_splits);
+
+/*
+ * sr_workspace_init -- zero the workspace (cudaMemsetAsync on `stream`). Call
+ * once after allocating it; afterwards every launch leaves the counters at zero.
+ */
+sr_status sr_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sr_decode_attention -- routed split-K decode attention for one layer step.
+ * Sink units (not listed in active_list): out[b, h] = v0[b, g] for every query
+ * head h of the group, bit for bit, with no cache read (README decode list,
+ * sink bypass). Active units: standard softmax attention over cache positions
+ * 0 .. L_b-1 (position 0 read from the cache), scale 1/sqrt(d):
+ *     out[b, h] = sum_j softmax_j(<q_h, K[b, g, j]> / sqrt(d)) V[b, g, j]
+ * (README decode list: tiled QK/PV, online softmax, Split-K with in-kernel
+ * reduction; pith.science review of arXiv 2604.16883, Figure 1 caption,
+ * eq. (1)). fp32 arithmetic on bf16 inputs; out is rounded to bf16 (RNE).
+ *
+ *   q           bf16 [B, Hq, d]
+ *   k_cache     bf16 [B, Hkv, Lmax, d]
+ *   v_cache     bf16 [B, Hkv, Lmax, d]
+ *   k0          bf16 [B, Hkv, d]; not read by this call (routing already used
+ *               it); may be NULL
+ *   v0          bf16 [B, Hkv, d]  cached position-0 value
+ *   seq_lens    int32 [B] device: valid positions per sequence, 1 <= L_b <= Lmax
+ *               (out of range: clamped, SR_DEVERR_SEQ_LEN). Positions >= L_b
+ *               are never used and may hold anything, NaN included.
+ *   active_list int32 [1 + B*Hkv] as written by sr_route (count, then strictly
+ *               ascending unit indices)
+ *   n_splits    0 = automatic: the active positions of all units are cut into
+ *               one contiguous share per persistent CTA (balanced across the
+ *               SMs, at least 256 positions each), decided on the device from
+ *               active_list and seq_lens. > 0: every active unit is cut into
+ *               exactly n_splits equal splits (<= SR_MAX_SPLITS).
+ *   out         bf16 [B, Hq, d]
+ *   workspace   device buffer of >= sr_decode_workspace_bytes(dims, n_splits)
+ *               bytes, 256-byte aligned, zeroed once by sr_workspace_init.
+ *               Two calls that overlap on the GPU must not share a workspace.
+ * Must run after sr_route on the same stream (or be ordered after it). One
+ * kernel launch. Errors: SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED,
+ * SR_ERR_WORKSPACE, SR_ERR_CUDA.
+ */
+sr_status sr_decode_attention(const sr_dims *dims, const void *q, const void *k_cache,
+                              const void *v_cache, const void *k0, const void *v0,
+                              const int32_t *seq_lens, const int32_t *active_list,
+                              int32_t n_splits, void *out, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/* Static description of a status code. */
+const char *sr_status_string(sr_status s);
+
+/*
+ * sr_get_device_error -- read the device error word of a workspace into *code
+ * (an OR of SR_DEVERR_* bits; 0 = none). Synchronises `stream`. Debug use.
+ */
+sr_status sr_get_device_error(const void *workspace, int32_t *code, void *stream);
+
+/* sr_clear_device_error -- reset the device error word to 0 (async on `stream`). */
+sr_status sr_clear_device_error(void *workspace, void *stream);
+
+/*
+ * sr_decode_grid_size -- number of persistent CTAs sr_decode_attention launches
+ * on the current device (its SM count times resident CTAs per SM). Returns 0
+ * when no device is usable.
+ */
+int32_t sr_decode_grid_size(void);
+
+/* Message of the last CUDA error seen by this library on this thread ("" if none). */
+const char *sr_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SINKROUTER_H */

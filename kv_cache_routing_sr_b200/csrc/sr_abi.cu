@@ -1,0 +1,155 @@
+// extern "C" entry points of libsinkrouter.so (declared in include/sinkrouter.h):
+// host-side validation, workspace layout and kernel dispatch. No function here
+// allocates device memory; every buffer is the caller's.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+#include <string>
+
+#include "sinkrouter.h"
+#include "sr_internal.h"
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+sr_status cuda_fail(cudaError_t e)
+{
+    g_last_cuda_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
+    return SR_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by both calls.
+sr_status check_dims(const sr_dims *d)
+{
+    if (!d)
+        return SR_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->n_kv_heads < 1 || d->n_q_heads < 1 || d->head_dim < 1 || d->max_seq_len < 1)
+        return SR_ERR_INVALID_ARG;
+    if (d->n_q_heads % d->n_kv_heads != 0)
+        return SR_ERR_INVALID_ARG;
+    if (d->head_dim != sr::kHeadDim)
+        return SR_ERR_UNSUPPORTED;
+    const int M = d->n_q_heads / d->n_kv_heads;
+    if (M != 1 && M != 2 && M != 4 && M != 8)
+        return SR_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * d->n_kv_heads > SR_MAX_UNITS)
+        return SR_ERR_UNSUPPORTED;
+    return SR_OK;
+}
+
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+} // namespace
+
+extern "C" {
+
+const char *sr_status_string(sr_status s)
+{
+    switch (s) {
+    case SR_OK:
+        return "SR_OK";
+    case SR_ERR_INVALID_ARG:
+        return "SR_ERR_INVALID_ARG: null/misaligned pointer or invalid size";
+    case SR_ERR_UNSUPPORTED:
+        return "SR_ERR_UNSUPPORTED: head_dim must be 128, group size 1/2/4/8, batch*kv_heads <= SR_MAX_UNITS";
+    case SR_ERR_WORKSPACE:
+        return "SR_ERR_WORKSPACE: workspace null, misaligned or too small";
+    case SR_ERR_CUDA:
+        return "SR_ERR_CUDA: a CUDA call failed (see sr_last_cuda_error)";
+    }
+    return "unknown sr_status";
+}
+
+const char *sr_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+sr_status sr_route(const sr_dims *dims, const void *q, const void *k0, float tau, uint8_t *route_mask,
+                   int32_t *active_list, void *stream)
+{
+    const sr_status st = check_dims(dims);
+    if (st != SR_OK)
+        return st;
+    if (!q || !k0 || !route_mask || !active_list || !aligned(q, 16) || !aligned(k0, 16) || !aligned(active_list, 4))
+        return SR_ERR_INVALID_ARG;
+    if (std::isnan(tau))
+        return SR_ERR_INVALID_ARG;
+    sr::RouteArgs a{q, k0, tau, route_mask, active_list, dims->batch, dims->n_q_heads, dims->n_kv_heads};
+    const cudaError_t e = sr::launch_route(a, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+size_t sr_decode_workspace_bytes(const sr_dims *dims, int32_t max_splits)
+{
+    if (check_dims(dims) != SR_OK || max_splits < 0 || max_splits > SR_MAX_SPLITS)
+        return 0;
+    const int U = dims->batch * dims->n_kv_heads;
+    const int M = dims->n_q_heads / dims->n_kv_heads;
+    int64_t slots = sr::slots_needed(U, 0);
+    if (max_splits > 0 && sr::slots_needed(U, max_splits) > slots)
+        slots = sr::slots_needed(U, max_splits);
+    return sr::workspace_layout(U, M, slots).total;
+}
+
+sr_status sr_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes == 0)
+        return SR_ERR_WORKSPACE;
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+sr_status sr_decode_attention(const sr_dims *dims, const void *q, const void *k_cache, const void *v_cache,
+                              const void *k0, const void *v0, const int32_t *seq_lens, const int32_t *active_list,
+                              int32_t n_splits, void *out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)k0; // routing already consumed it; the scan reads position 0 from the cache
+    const sr_status st = check_dims(dims);
+    if (st != SR_OK)
+        return st;
+    if (!q || !k_cache || !v_cache || !v0 || !seq_lens || !active_list || !out)
+        return SR_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(v0, 16) ||
+        !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(active_list, 4))
+        return SR_ERR_INVALID_ARG;
+    if (n_splits < 0 || n_splits > SR_MAX_SPLITS)
+        return SR_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256))
+        return SR_ERR_WORKSPACE;
+    const int U = dims->batch * dims->n_kv_heads;
+    const int M = dims->n_q_heads / dims->n_kv_heads;
+    const sr::WorkspaceLayout ws = sr::workspace_layout(U, M, sr::slots_needed(U, n_splits));
+    if (workspace_bytes < ws.total)
+        return SR_ERR_WORKSPACE;
+    sr::DecodeArgs a{q,   k_cache,      v_cache,         v0,         seq_lens,         active_list,
+                     out, workspace,    ws,              dims->batch, dims->n_q_heads, dims->n_kv_heads,
+                     dims->max_seq_len, n_splits};
+    const cudaError_t e = sr::launch_decode(a, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+sr_status sr_get_device_error(const void *workspace, int32_t *code, void *stream)
+{
+    if (!workspace || !aligned(workspace, 256))
+        return SR_ERR_WORKSPACE;
+    if (!code)
+        return SR_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemcpyAsync(code, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, as_stream(stream));
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+sr_status sr_clear_device_error(void *workspace, void *stream)
+{
+    if (!workspace || !aligned(workspace, 256))
+        return SR_ERR_WORKSPACE;
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int32_t), as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+int32_t sr_decode_grid_size(void) { return sr::decode_grid_size(); }
+
+} // extern "C"

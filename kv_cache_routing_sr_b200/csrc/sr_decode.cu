@@ -1,0 +1,805 @@
+// Split-K decode attention over the active units, with the sink bypass and the
+// cross-split reduction in the same persistent kernel.
+//
+// Method: SinkRouter README (github.com/streamer-AP/SinkRouter), decode-time
+// procedure list -- sink groups return the position-0 value, active groups run
+// tiled QK / PV with online softmax, Split-K over the context and an in-kernel
+// reduction; sota2 summary, Abstract -- decode attention is memory-bound on the
+// KV-cache read. Output definition: pith.science review of arXiv 2604.16883,
+// Figure 1 caption, eq. (1) (attention-weighted sum of cached values).
+//
+// Design (B200, sm_100a):
+//  * One persistent CTA per SM: 4 consumer warps + 1 producer warp. The grid
+//    never depends on the route result, so the launch needs no host sync; each
+//    CTA reads the active list and seq_lens and derives its share of the work.
+//  * Automatic splits: the active positions of all units are concatenated and
+//    cut into one contiguous chunk per CTA (rounded to whole tiles, >= 256
+//    positions), so every SM streams the same number of bytes whatever the mix
+//    of unit lengths. A chunk may cover the end of one unit and the start of
+//    the next; each (CTA, unit) overlap is one split.
+//  * The producer lane walks its splits tile by tile and issues 3-D TMA loads
+//    (two 128-byte-wide boxes for K, two for V, 128B swizzle) into a ring of
+//    shared-memory stages, each guarded by a full/empty mbarrier pair. A small
+//    header in each stage tells the consumers which unit / rows the tile holds.
+//  * Each consumer warp owns 16*RB rows of every tile. S^T = K_tile * Q^T on
+//    bf16 mma.sync m16n8k16 (positions on M, the group's query heads on N;
+//    the tile is read once for all M heads), online softmax in fp32 with exp2,
+//    P^T moved into the B-operand layout with movmatrix, O^T += V^T * P^T with
+//    ldmatrix.trans. The contraction is tiny (M <= 8 heads), so the tensor
+//    cores only serve to keep the issue rate far below the HBM stream rate.
+//  * At the end of a split the four warps merge their (m, l, O) in shared
+//    memory, write one fp32 partial, and count it on the unit's arrival
+//    counter. The CTA that brings the counter to the unit's split count merges
+//    all partials of the unit in a fixed order, writes the bf16 output and
+//    resets the counter (nobody ever waits for another CTA).
+//  * Sink units: while the first tiles are in flight, the consumer warps copy
+//    v0 into the output of every unit absent from the active list.
+//  * Every wait is bounded in time; a timeout sets a device error bit and the
+//    CTA leaves after its in-flight copies have landed.
+#include <climits>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "sinkrouter.h"
+#include "sr_internal.h"
+#include "sr_ptx.cuh"
+
+#ifndef SR_DECODE_RB
+#define SR_DECODE_RB 1 // row blocks of 16 per consumer warp and tile
+#endif
+#ifndef SR_DECODE_STAGES
+#define SR_DECODE_STAGES 4
+#endif
+
+namespace sr {
+namespace {
+
+constexpr int kCWarps = 4;
+constexpr int kThreads = 32 * (kCWarps + 1);
+constexpr long long kMinChunk = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull; // 2 s: far above any legitimate wait
+constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
+
+struct alignas(16) TileHdr {
+    int32_t unit;       // flat unit b*Hkv+g
+    int32_t pos0;       // unit-local position of tile row 0
+    int32_t nvalid;     // rows of the tile inside the split (0: empty split)
+    int32_t flags;      // kFirst | kLast | kEnd
+    int32_t slot;       // partial slot of this split
+    int32_t nseg;       // splits of this unit
+    int32_t slot_first; // slot of the unit's first split (its slots are consecutive)
+    int32_t pad;
+};
+
+struct Misc {
+    int abort_flag;
+    int is_last;
+    int i0;
+    int pad;
+    long long s0;
+    long long wsum[kCWarps + 1];
+};
+
+struct Params {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *v0;
+    const int32_t *seq_lens;
+    const int32_t *active;
+    __nv_bfloat16 *out;
+    int32_t *err;
+    int32_t *cnt;
+    float *part_o;
+    float2 *part_ml;
+    int B, Hq, Hkv, M, Lmax, n_splits;
+};
+
+template <int RB, int STAGES> struct Cfg {
+    static constexpr int BN = 16 * RB * kCWarps; // positions per tile
+    static constexpr int HALF = BN * 128;        // one [BN x 64] bf16 box
+    static constexpr int STAGE = 4 * HALF;       // K lo, K hi, V lo, V hi
+    static constexpr int QBYTES = kMaxGroup * kHeadDim * 2;
+    static constexpr int OFF_Q = STAGES * STAGE;
+    static constexpr int OFF_COMB = OFF_Q + STAGES * QBYTES;
+    static constexpr int OFF_ML = OFF_COMB + kCWarps * kMaxGroup * kHeadDim * 4;
+    static constexpr int OFF_HDR = OFF_ML + kCWarps * kMaxGroup * 8;
+    static constexpr int OFF_BAR = OFF_HDR + STAGES * (int)sizeof(TileHdr);
+    static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
+    static constexpr int OFF_BITMAP = OFF_MISC + 128;
+    static constexpr int BYTES = OFF_BITMAP + SR_MAX_UNITS / 8;
+    static constexpr int ALLOC = BYTES + 1024; // room to align the base to 1024 B
+    static_assert(sizeof(Misc) <= 128, "misc block");
+    static_assert(BN <= 256, "TMA box rows");
+    static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (*abort_flag)
+            return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Valid length of the i-th active entry, or 0 when the entry is skipped
+// (index out of range or list not strictly ascending). Lengths are clamped to
+// [1, Lmax]. Pure function of global data, so every thread gets the same answer.
+__device__ __forceinline__ int active_len(const Params &p, int i, int U, int &u, int &errbits)
+{
+    u = __ldg(p.active + 1 + i);
+    const int prev = (i > 0) ? __ldg(p.active + i) : -1;
+    if (u < 0 || u >= U || u <= prev) {
+        errbits |= SR_DEVERR_ACTIVE_LIST;
+        return 0;
+    }
+    int L = __ldg(p.seq_lens + u / p.Hkv);
+    if (L < 1 || L > p.Lmax) {
+        errbits |= SR_DEVERR_SEQ_LEN;
+        L = L < 1 ? 1 : p.Lmax;
+    }
+    return L;
+}
+
+// Inclusive block-wide prefix of a 64-bit value; *total receives the block sum.
+__device__ __forceinline__ long long block_scan(long long x, Misc *misc, long long *total)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long v = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o)
+            v += y;
+    }
+    if (lane == 31)
+        misc->wsum[warp] = v;
+    __syncthreads();
+    long long before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kCWarps + 1; ++w) {
+        const long long s = misc->wsum[w];
+        before += (w < warp) ? s : 0;
+        all += s;
+    }
+    __syncthreads();
+    *total = all;
+    return before + v;
+}
+
+template <int RB, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p)
+{
+    using C = Cfg<RB, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    TileHdr *hdr = reinterpret_cast<TileHdr *>(smem + C::OFF_HDR);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR); // full[S], empty[S], consumer sync
+    Misc *misc = reinterpret_cast<Misc *>(smem + C::OFF_MISC);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + C::OFF_BITMAP);
+    float *comb = reinterpret_cast<float *>(smem + C::OFF_COMB);
+    float2 *mlsm = reinterpret_cast<float2 *>(smem + C::OFF_ML);
+    volatile int *abort_flag = &misc->abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int U = p.B * p.Hkv;
+    const int M = p.M;
+    const uint32_t full0 = smem_u32(&bars[0]);
+    const uint32_t empty0 = smem_u32(&bars[STAGES]);
+    const uint32_t cbar = smem_u32(&bars[2 * STAGES]);
+
+    // ---------------------------------------------------------------- prologue
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, kCWarps);
+        }
+        mbar_init(cbar, kCWarps);
+        fence_mbar_init();
+        misc->abort_flag = 0;
+        misc->is_last = 0;
+        misc->i0 = INT_MAX;
+        misc->s0 = 0;
+    }
+    for (int w = tid; w < (U + 31) / 32; w += kThreads)
+        bitmap[w] = 0;
+    __syncthreads();
+
+    int errbits = 0;
+    int n = __ldg(p.active);
+    if (n < 0 || n > U) {
+        errbits |= SR_DEVERR_ACTIVE_LIST;
+        n = n < 0 ? 0 : U;
+    }
+    long long local = 0;
+    for (int i = tid; i < n; i += kThreads) {
+        int u;
+        const int L = active_len(p, i, U, u, errbits);
+        if (L > 0) {
+            atomicOr(&bitmap[u >> 5], 1u << (u & 31));
+            local += L;
+        }
+    }
+    long long P;
+    (void)block_scan(local, misc, &P);
+    if (errbits && blockIdx.x == 0)
+        atomicOr(p.err, errbits);
+
+    const int G = gridDim.x;
+    long long chunk = 1, r0 = 0, r1 = 0;
+    if (p.n_splits == 0 && P > 0) {
+        chunk = (P + G - 1) / G;
+        chunk = (chunk + C::BN - 1) / C::BN * C::BN;
+        chunk = chunk < kMinChunk ? kMinChunk : chunk;
+        r0 = (long long)blockIdx.x * chunk;
+        r1 = r0 + chunk < P ? r0 + chunk : P;
+        if (r0 < P) { // find the active entry whose positions contain r0
+            long long carry = 0;
+            for (int base = 0; base < n; base += kThreads) {
+                const int i = base + tid;
+                int L = 0, u, dummy = 0;
+                if (i < n)
+                    L = active_len(p, i, U, u, dummy);
+                long long tot;
+                const long long incl = block_scan(L, misc, &tot);
+                const long long S = carry + incl - L;
+                if (i < n && L > 0 && S <= r0 && r0 < S + L) {
+                    misc->i0 = i;
+                    misc->s0 = S;
+                }
+                carry += tot;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- producer
+    if (warp == kCWarps) {
+        if (lane != 0)
+            return;
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        const uint64_t pol = l2_policy_evict_first();
+        int stage = 0;
+        uint32_t ph = 0;
+        int issued_parity[STAGES];
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s)
+            issued_parity[s] = -1;
+        bool ok = true;
+
+        auto emit = [&](const TileHdr &h, const void *qsrc, uint32_t qbytes) -> bool {
+            if (!wait_bar(empty0 + 8 * stage, ph ^ 1, abort_flag))
+                return false;
+            hdr[stage] = h;
+            const uint32_t fb = full0 + 8 * stage;
+            const uint32_t bytes = (h.nvalid > 0 ? (uint32_t)C::STAGE : 0u) + qbytes;
+            if (bytes) {
+                mbar_arrive_expect_tx(fb, bytes);
+                if (h.nvalid > 0) {
+                    const uint32_t sb = smem_u32(smem + stage * C::STAGE);
+                    tma_load_3d(sb, &tmK, fb, 0, h.pos0, h.unit, pol);
+                    tma_load_3d(sb + C::HALF, &tmK, fb, 64, h.pos0, h.unit, pol);
+                    tma_load_3d(sb + 2 * C::HALF, &tmV, fb, 0, h.pos0, h.unit, pol);
+                    tma_load_3d(sb + 3 * C::HALF, &tmV, fb, 64, h.pos0, h.unit, pol);
+                }
+                if (qbytes)
+                    bulk_load(smem_u32(smem + C::OFF_Q + stage * C::QBYTES), qsrc, qbytes, fb);
+                issued_parity[stage] = (int)ph;
+            } else {
+                mbar_arrive(fb);
+            }
+            if (++stage == STAGES) {
+                stage = 0;
+                ph ^= 1;
+            }
+            return true;
+        };
+
+        auto emit_split = [&](int u, long long b0, long long e0, int slot, int nseg, int slot_first) -> bool {
+            const long long len = e0 - b0;
+            const long long ntiles = len > 0 ? (len + C::BN - 1) / C::BN : 1;
+            const int sb = u / p.Hkv, sg = u - sb * p.Hkv;
+            const __nv_bfloat16 *qsrc = p.q + ((size_t)sb * p.Hq + (size_t)sg * M) * kHeadDim;
+            for (long long t = 0; t < ntiles; ++t) {
+                TileHdr h;
+                h.unit = u;
+                h.pos0 = (int)(b0 + t * C::BN);
+                const long long rem = e0 - h.pos0;
+                h.nvalid = len > 0 ? (int)(rem < C::BN ? rem : C::BN) : 0;
+                h.flags = (t == 0 ? kFirst : 0) | (t == ntiles - 1 ? kLast : 0);
+                h.slot = slot;
+                h.nseg = nseg;
+                h.slot_first = slot_first;
+                h.pad = 0;
+                const uint32_t qb = (t == 0 && len > 0) ? (uint32_t)(M * kHeadDim * 2) : 0u;
+                if (!emit(h, qsrc, qb))
+                    return false;
+            }
+            return true;
+        };
+
+        if (p.n_splits == 0) {
+            if (P > 0 && r0 < P) {
+                int i = misc->i0;
+                long long S = misc->s0;
+                while (ok && i < n && S < r1) {
+                    int u, dummy = 0;
+                    const int L = active_len(p, i, U, u, dummy);
+                    if (L > 0) {
+                        const long long b0 = (r0 > S ? r0 : S) - S;
+                        const long long e0 = (r1 < S + L ? r1 : S + L) - S;
+                        const long long cf = S / chunk, cl = (S + L - 1) / chunk;
+                        ok = emit_split(u, b0, e0, (int)blockIdx.x + i, (int)(cl - cf + 1), (int)cf + i);
+                    }
+                    S += L;
+                    ++i;
+                }
+            }
+        } else {
+            const int ns = p.n_splits;
+            for (long long j = blockIdx.x; ok && j < (long long)n * ns; j += G) {
+                const int i = (int)(j / ns), s = (int)(j % ns);
+                int u, dummy = 0;
+                const int L = active_len(p, i, U, u, dummy);
+                if (L == 0)
+                    continue;
+                const long long b0 = (long long)s * L / ns, e0 = (long long)(s + 1) * L / ns;
+                ok = emit_split(u, b0, e0, (int)j, ns, i * ns);
+            }
+        }
+        if (ok) {
+            TileHdr h{};
+            h.unit = -1;
+            h.flags = kEnd;
+            ok = emit(h, nullptr, 0);
+        }
+        if (!ok) {
+            atomicOr(p.err, SR_DEVERR_TIMEOUT);
+            // Let every copy still in flight land before this CTA can exit.
+            volatile int never = 0;
+            for (int s = 0; s < STAGES; ++s)
+                if (issued_parity[s] >= 0)
+                    (void)wait_bar(full0 + 8 * s, (uint32_t)issued_parity[s], &never);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int w = warp;
+    const int g = lane >> 2, t = lane & 3;
+    const int mi = lane >> 3, ri = lane & 7;
+    const int ctid = tid; // 0 .. 32*kCWarps-1
+
+    // Sink bypass: out[b, h] = v0[b, g] for every unit not in the active list.
+    {
+        const int gw = blockIdx.x * kCWarps + w, nw = gridDim.x * kCWarps;
+        for (int u = gw; u < U; u += nw) {
+            if (bitmap[u >> 5] & (1u << (u & 31)))
+                continue;
+            const int b = u / p.Hkv, gg = u - b * p.Hkv;
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.v0 + (size_t)u * kHeadDim) + (lane & 15));
+            for (int e = lane; e < M * 16; e += 32) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + (e >> 4)) * kHeadDim);
+                dst[e & 15] = v;
+            }
+        }
+    }
+
+    const uint32_t sbase = smem_u32(smem);
+    uint32_t rowK[RB], rowV[RB];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+        const int r = (w * RB + rb) * 16;
+        rowK[rb] = (uint32_t)(r + ri + 8 * (mi & 1)) * 128u;
+        rowV[rb] = (uint32_t)(r + ri + 8 * (mi >> 1)) * 128u;
+    }
+    const int my_row0 = w * RB * 16;
+
+    float o[8][4];
+    float mrun[2], lrun[2];
+    uint32_t qf[8][2];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        qf[j][0] = qf[j][1] = 0u;
+    }
+    mrun[0] = mrun[1] = -INFINITY;
+    lrun[0] = lrun[1] = 0.f;
+
+    int stage = 0;
+    uint32_t ph = 0, cph = 0;
+    bool ok = true;
+
+    auto cbar_sync = [&]() -> bool {
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(cbar);
+        bool r = wait_bar(cbar, cph, abort_flag);
+        cph ^= 1;
+        return __all_sync(0xffffffffu, r);
+    };
+
+    for (;;) {
+        if (!__all_sync(0xffffffffu, wait_bar(full0 + 8 * stage, ph, abort_flag))) {
+            ok = false;
+            break;
+        }
+        const TileHdr h = hdr[stage];
+        if (h.flags & kEnd)
+            break;
+        const uint32_t st = sbase + stage * C::STAGE;
+        if (h.flags & kFirst) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+            mrun[0] = mrun[1] = -INFINITY;
+            lrun[0] = lrun[1] = 0.f;
+            if (h.nvalid > 0) {
+                const uint32_t *qs = reinterpret_cast<const uint32_t *>(smem + C::OFF_Q + stage * C::QBYTES);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    qf[ks][0] = (g < M) ? qs[g * 64 + ks * 8 + t] : 0u;
+                    qf[ks][1] = (g < M) ? qs[g * 64 + ks * 8 + 4 + t] : 0u;
+                }
+            }
+        }
+
+        if (h.nvalid > my_row0) {
+            if (h.nvalid < my_row0 + RB * 16) {
+                // Rows past the split may be padding (even NaN): zero this
+                // warp's V rows there so that P = 0 contributes exactly 0.
+                const int z0 = h.nvalid, nz = my_row0 + RB * 16 - z0;
+                for (int e = lane; e < nz * 16; e += 32) {
+                    const int row = z0 + (e >> 4), c = e & 15;
+                    uint4 *dst = reinterpret_cast<uint4 *>(smem + stage * C::STAGE + (2 + (c >> 3)) * C::HALF +
+                                                           row * 128 + (c & 7) * 16);
+                    *dst = make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+
+            // S^T[16 rows x 8 heads] per row block, two accumulators per block.
+            float sacc[RB][4];
+            {
+                float sa[RB][4], sb[RB][4];
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        sa[rb][e] = sb[rb][e] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kb = st + (uint32_t)(ks >> 2) * C::HALF;
+                    const uint32_t cx = (uint32_t)(((ks & 3) * 2 + (mi >> 1)) ^ ri) << 4;
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        uint32_t a[4];
+                        ldmatrix_x4(a, kb + rowK[rb] + cx);
+                        if (ks & 1)
+                            mma_bf16_16816(sb[rb], a, qf[ks][0], qf[ks][1]);
+                        else
+                            mma_bf16_16816(sa[rb], a, qf[ks][0], qf[ks][1]);
+                    }
+                }
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int row = my_row0 + rb * 16 + g + (e >> 1) * 8;
+                        sacc[rb][e] = (row < h.nvalid) ? (sa[rb][e] + sb[rb][e]) * kScaleLog2 : -INFINITY;
+                    }
+            }
+
+            // Online softmax (log2 domain); lane holds heads 2t and 2t+1.
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                mx0 = fmaxf(mx0, fmaxf(sacc[rb][0], sacc[rb][2]));
+                mx1 = fmaxf(mx1, fmaxf(sacc[rb][1], sacc[rb][3]));
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            }
+            const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
+            const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
+            const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+            const float al0 = exp2f(mrun[0] - mu0), al1 = exp2f(mrun[1] - mu1);
+            mrun[0] = mn0;
+            mrun[1] = mn1;
+            float ps0 = 0.f, ps1 = 0.f;
+            uint32_t pf[RB][2];
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb) {
+                const float p0 = exp2f(sacc[rb][0] - mu0), p1 = exp2f(sacc[rb][1] - mu1);
+                const float p2 = exp2f(sacc[rb][2] - mu0), p3 = exp2f(sacc[rb][3] - mu1);
+                ps0 += p0 + p2;
+                ps1 += p1 + p3;
+                pf[rb][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+                pf[rb][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+            }
+            lrun[0] = lrun[0] * al0 + ps0;
+            lrun[1] = lrun[1] * al1 + ps1;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                o[j][0] *= al0;
+                o[j][1] *= al1;
+                o[j][2] *= al0;
+                o[j][3] *= al1;
+            }
+
+            // O^T[128 x 8 heads] += V^T * P^T, 16 head-dim rows per MMA.
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t vb = st + (uint32_t)(2 + (j >> 2)) * C::HALF;
+                const uint32_t cx = (uint32_t)(((j & 3) * 2 + (mi & 1)) ^ ri) << 4;
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(a, vb + rowV[rb] + cx);
+                    mma_bf16_16816(o[j], a, pf[rb][0], pf[rb][1]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(empty0 + 8 * stage);
+
+        if (h.flags & kLast) {
+            // ---- merge the four warps' states into one partial of this split
+            float l0 = lrun[0], l1 = lrun[1];
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+            }
+            if (g == 0) {
+                mlsm[w * kMaxGroup + 2 * t] = make_float2(mrun[0], l0);
+                mlsm[w * kMaxGroup + 2 * t + 1] = make_float2(mrun[1], l1);
+            }
+            if (!(ok = cbar_sync()))
+                break;
+            float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+            for (int ww = 0; ww < kCWarps; ++ww) {
+                M0 = fmaxf(M0, mlsm[ww * kMaxGroup + 2 * t].x);
+                M1 = fmaxf(M1, mlsm[ww * kMaxGroup + 2 * t + 1].x);
+            }
+            const float f0 = (M0 == -INFINITY) ? 0.f : exp2f(mrun[0] - M0);
+            const float f1 = (M1 == -INFINITY) ? 0.f : exp2f(mrun[1] - M1);
+            float *cw = comb + w * (kMaxGroup * kHeadDim);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int d0 = 16 * j + g;
+                if (2 * t < M) {
+                    cw[(2 * t) * kHeadDim + d0] = o[j][0] * f0;
+                    cw[(2 * t) * kHeadDim + d0 + 8] = o[j][2] * f0;
+                }
+                if (2 * t + 1 < M) {
+                    cw[(2 * t + 1) * kHeadDim + d0] = o[j][1] * f1;
+                    cw[(2 * t + 1) * kHeadDim + d0 + 8] = o[j][3] * f1;
+                }
+            }
+            if (!(ok = cbar_sync()))
+                break;
+            float *po = p.part_o + (size_t)h.slot * M * kHeadDim;
+            for (int idx = ctid; idx < M * 32; idx += 32 * kCWarps) {
+                const int head = idx >> 5, d4 = (idx & 31) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int ww = 0; ww < kCWarps; ++ww) {
+                    const float4 x =
+                        *reinterpret_cast<const float4 *>(comb + ww * (kMaxGroup * kHeadDim) + head * kHeadDim + d4);
+                    acc.x += x.x, acc.y += x.y, acc.z += x.z, acc.w += x.w;
+                }
+                __stcg(reinterpret_cast<float4 *>(po + head * kHeadDim + d4), acc);
+            }
+            if (ctid < M) {
+                float Mh = -INFINITY;
+#pragma unroll
+                for (int ww = 0; ww < kCWarps; ++ww)
+                    Mh = fmaxf(Mh, mlsm[ww * kMaxGroup + ctid].x);
+                float Lh = 0.f;
+                if (Mh != -INFINITY) {
+#pragma unroll
+                    for (int ww = 0; ww < kCWarps; ++ww) {
+                        const float2 x = mlsm[ww * kMaxGroup + ctid];
+                        if (x.x != -INFINITY)
+                            Lh += x.y * exp2f(x.x - Mh);
+                    }
+                }
+                __stcg(p.part_ml + (size_t)h.slot * M + ctid, make_float2(Mh, Lh));
+            }
+            __threadfence();
+            if (!(ok = cbar_sync()))
+                break;
+            if (ctid == 0)
+                misc->is_last = (atomicAdd(p.cnt + h.unit, 1) == h.nseg - 1) ? 1 : 0;
+            if (!(ok = cbar_sync()))
+                break;
+            if (misc->is_last) {
+                // ---- last split of the unit to finish: merge all its partials
+                __threadfence();
+                const int b = h.unit / p.Hkv, gg = h.unit - b * p.Hkv;
+                for (int idx = ctid; idx < M * 32; idx += 32 * kCWarps) {
+                    const int head = idx >> 5, d4 = (idx & 31) * 4;
+                    float m = -INFINITY, l = 0.f;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int j = 0; j < h.nseg; ++j) {
+                        const size_t sl = (size_t)(h.slot_first + j) * M + head;
+                        const float2 x = __ldcg(p.part_ml + sl);
+                        const float4 y = __ldcg(reinterpret_cast<const float4 *>(p.part_o + sl * kHeadDim + d4));
+                        if (x.x == -INFINITY)
+                            continue;
+                        const float mn = fmaxf(m, x.x);
+                        const float a = exp2f(m - mn), c = exp2f(x.x - mn);
+                        l = l * a + x.y * c;
+                        acc.x = acc.x * a + y.x * c;
+                        acc.y = acc.y * a + y.y * c;
+                        acc.z = acc.z * a + y.z * c;
+                        acc.w = acc.w * a + y.w * c;
+                        m = mn;
+                    }
+                    const float inv = 1.f / l;
+                    uint2 packed;
+                    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+                    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+                    *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim + d4) =
+                        packed;
+                }
+                if (ctid == 0)
+                    p.cnt[h.unit] = 0;
+            }
+        }
+        if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+        }
+    }
+    if (!ok && lane == 0)
+        atomicOr(p.err, SR_DEVERR_TIMEOUT);
+}
+
+// ---- host side ------------------------------------------------------------------------
+
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const Params);
+
+struct DeviceInfo {
+    int sms = 0;
+    int grid = 0;
+    bool configured = false;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3-D view [units][Lmax][128] of a bf16 cache; a box is 64 columns (128 bytes,
+// swizzled 128B) by `rows` positions of one unit. Rows past Lmax read as zero.
+bool make_cache_map(CUtensorMap *map, const void *base, int units, int lmax, int rows)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)lmax, (cuuint64_t)units};
+    cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)lmax * kHeadDim * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+using DecodeCfg = Cfg<SR_DECODE_RB, SR_DECODE_STAGES>;
+
+cudaError_t configure(int dev, DeviceInfo &info)
+{
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (info.configured)
+        return cudaSuccess;
+    cudaError_t e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
+    KernelFn k = decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg::ALLOC);
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, DecodeCfg::ALLOC);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        return cudaErrorInvalidConfiguration;
+    info.grid = info.sms * per_sm;
+    if (info.grid > kAutoGridCap)
+        info.grid = kAutoGridCap;
+    info.configured = true;
+    return cudaSuccess;
+}
+
+cudaError_t device_info(DeviceInfo **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    e = configure(dev, g_dev[dev]);
+    *out = &g_dev[dev];
+    return e;
+}
+
+} // namespace
+
+int decode_grid_size()
+{
+    DeviceInfo *info = nullptr;
+    if (device_info(&info) != cudaSuccess)
+        return 0;
+    return info->grid;
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
+{
+    DeviceInfo *info = nullptr;
+    cudaError_t e = device_info(&info);
+    if (e != cudaSuccess)
+        return e;
+    const int U = a.batch * a.n_kv_heads;
+    CUtensorMap tmK, tmV;
+    if (!make_cache_map(&tmK, a.k_cache, U, a.max_seq_len, DecodeCfg::BN) ||
+        !make_cache_map(&tmV, a.v_cache, U, a.max_seq_len, DecodeCfg::BN))
+        return cudaErrorInvalidValue;
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    Params p;
+    p.q = static_cast<const __nv_bfloat16 *>(a.q);
+    p.v0 = static_cast<const __nv_bfloat16 *>(a.v0);
+    p.seq_lens = a.seq_lens;
+    p.active = a.active_list;
+    p.out = static_cast<__nv_bfloat16 *>(a.out);
+    p.err = reinterpret_cast<int32_t *>(ws + a.ws.err_off);
+    p.cnt = reinterpret_cast<int32_t *>(ws + a.ws.cnt_off);
+    p.part_o = reinterpret_cast<float *>(ws + a.ws.part_o_off);
+    p.part_ml = reinterpret_cast<float2 *>(ws + a.ws.part_ml_off);
+    p.B = a.batch;
+    p.Hq = a.n_q_heads;
+    p.Hkv = a.n_kv_heads;
+    p.M = a.n_q_heads / a.n_kv_heads;
+    p.Lmax = a.max_seq_len;
+    p.n_splits = a.n_splits;
+    decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES><<<info->grid, kThreads, DecodeCfg::ALLOC, stream>>>(tmK, tmV, p);
+    return cudaGetLastError();
+}
+
+} // namespace sr

@@ -1,0 +1,66 @@
+// Internal interfaces between the C-ABI layer (sr_abi.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sr {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxGroup = 8;      // query heads per KV head handled by one n8 MMA tile
+constexpr int kAutoGridCap = 1024; // persistent CTAs never exceed this (sizes the workspace)
+
+// Workspace layout: [error word | per-unit arrival counters | partial O | partial (m, l)].
+struct WorkspaceLayout {
+    size_t err_off = 0;
+    size_t cnt_off = 256;
+    size_t part_o_off = 0;
+    size_t part_ml_off = 0;
+    size_t total = 0;
+    int64_t slots = 0;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Partial slots a launch may touch: automatic splits use slot = cta + active
+// index (< grid + units); forced splits use active index * n_splits + split.
+inline int64_t slots_needed(int units, int n_splits)
+{
+    return n_splits > 0 ? (int64_t)units * n_splits : (int64_t)kAutoGridCap + units;
+}
+
+inline WorkspaceLayout workspace_layout(int units, int group, int64_t slots)
+{
+    WorkspaceLayout w;
+    w.slots = slots;
+    w.part_o_off = align_up(w.cnt_off + sizeof(int32_t) * (size_t)units, 256);
+    w.part_ml_off = align_up(w.part_o_off + sizeof(float) * (size_t)slots * group * kHeadDim, 256);
+    w.total = align_up(w.part_ml_off + 2 * sizeof(float) * (size_t)slots * group, 256);
+    return w;
+}
+
+struct RouteArgs {
+    const void *q;
+    const void *k0;
+    float tau;
+    uint8_t *mask;
+    int32_t *active;
+    int batch, n_q_heads, n_kv_heads;
+};
+
+struct DecodeArgs {
+    const void *q, *k_cache, *v_cache, *v0;
+    const int32_t *seq_lens, *active_list;
+    void *out;
+    void *workspace;
+    WorkspaceLayout ws;
+    int batch, n_q_heads, n_kv_heads, max_seq_len, n_splits;
+};
+
+cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+// Persistent CTAs of the decode kernel on the current device (0 on error).
+int decode_grid_size();
+
+} // namespace sr

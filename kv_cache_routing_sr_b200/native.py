@@ -1,0 +1,194 @@
+"""ctypes binding of libsinkrouter.so (the C ABI in include/sinkrouter.h).
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels. torch provides device memory and the current stream. There is no
+CPU fallback: a missing or unloadable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIBRARY = _build.LIBRARY
+
+SR_OK, SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_WORKSPACE, SR_ERR_CUDA = range(5)
+SR_DEVERR_SEQ_LEN, SR_DEVERR_ACTIVE_LIST, SR_DEVERR_TIMEOUT = 1, 2, 4
+SR_MAX_UNITS = 16384
+SR_MAX_SPLITS = 4096
+HEAD_DIM = 128
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("max_seq_len", ctypes.c_int32)]
+
+
+class SinkRouterError(RuntimeError):
+    def __init__(self, fn: str, status: int, lib):
+        msg = lib.sr_status_string(status).decode()
+        if status == SR_ERR_CUDA:
+            msg += " -- " + lib.sr_last_cuda_error().decode()
+        super().__init__(f"{fn}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_decode_attention",
+           "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
+           "sr_last_cuda_error"]
+
+
+def load(path: str = LIBRARY):
+    """Load (once) and type the library. Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libsinkrouter.so not found at {path}: build it with "
+                           "`python -m kv_cache_routing_sr_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, i32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    dp = ctypes.POINTER(Dims)
+    lib.sr_route.argtypes = [dp, vp, vp, ctypes.c_float, vp, vp, vp]
+    lib.sr_route.restype = ctypes.c_int
+    lib.sr_decode_workspace_bytes.argtypes = [dp, i32]
+    lib.sr_decode_workspace_bytes.restype = u64
+    lib.sr_workspace_init.argtypes = [vp, u64, vp]
+    lib.sr_workspace_init.restype = ctypes.c_int
+    lib.sr_decode_attention.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, u64, vp]
+    lib.sr_decode_attention.restype = ctypes.c_int
+    lib.sr_status_string.argtypes = [ctypes.c_int]
+    lib.sr_status_string.restype = ctypes.c_char_p
+    lib.sr_get_device_error.argtypes = [vp, ctypes.POINTER(i32), vp]
+    lib.sr_get_device_error.restype = ctypes.c_int
+    lib.sr_clear_device_error.argtypes = [vp, vp]
+    lib.sr_clear_device_error.restype = ctypes.c_int
+    lib.sr_decode_grid_size.argtypes = []
+    lib.sr_decode_grid_size.restype = i32
+    lib.sr_last_cuda_error.argtypes = []
+    lib.sr_last_cuda_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != SR_OK:
+        raise SinkRouterError(fn, status, load())
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def dims_of(batch: int, n_q_heads: int, n_kv_heads: int, max_seq_len: int, head_dim: int = HEAD_DIM) -> Dims:
+    return Dims(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len)
+
+
+def workspace_bytes(batch, n_q_heads, n_kv_heads, max_seq_len, max_splits: int = 0) -> int:
+    d = dims_of(batch, n_q_heads, n_kv_heads, max_seq_len)
+    n = load().sr_decode_workspace_bytes(ctypes.byref(d), int(max_splits))
+    if n == 0:
+        raise ValueError("unsupported dims or max_splits for the decode workspace")
+    return int(n)
+
+
+class Workspace:
+    """A zero-initialised decode workspace in torch-allocated device memory."""
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, max_seq_len, max_splits: int = 0, device=None):
+        self.nbytes = workspace_bytes(batch, n_q_heads, n_kv_heads, max_seq_len, max_splits)
+        self.buffer = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        off = (-self.buffer.data_ptr()) % 256
+        self.view = self.buffer[off:off + self.nbytes]
+        _check("sr_workspace_init", load().sr_workspace_init(ctypes.c_void_p(self.view.data_ptr()),
+                                                             self.nbytes, _stream()))
+
+    @property
+    def ptr(self) -> int:
+        return self.view.data_ptr()
+
+    def device_error(self) -> int:
+        code = ctypes.c_int32(0)
+        _check("sr_get_device_error", load().sr_get_device_error(ctypes.c_void_p(self.ptr),
+                                                                 ctypes.byref(code), _stream()))
+        return int(code.value)
+
+    def clear_device_error(self):
+        _check("sr_clear_device_error", load().sr_clear_device_error(ctypes.c_void_p(self.ptr), _stream()))
+
+
+def route(q: torch.Tensor, k0: torch.Tensor, tau: float, route_mask=None, active_list=None, stream=None):
+    """sr_route: returns (route_mask uint8 [B*Hkv], active_list int32 [1+B*Hkv])."""
+    B, Hq, d = q.shape
+    Hkv = k0.shape[1]
+    if route_mask is None:
+        route_mask = torch.empty(B * Hkv, dtype=torch.uint8, device=q.device)
+    if active_list is None:
+        active_list = torch.empty(1 + B * Hkv, dtype=torch.int32, device=q.device)
+    dims = dims_of(B, Hq, Hkv, 1, d)
+    st = load().sr_route(ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k0, "k0", torch.bfloat16),
+                         float(tau), _dev(route_mask, "route_mask", torch.uint8),
+                         _dev(active_list, "active_list", torch.int32), _stream(stream))
+    _check("sr_route", st)
+    return route_mask, active_list
+
+
+def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=None, n_splits: int = 0,
+                     workspace: Workspace | None = None, stream=None):
+    """sr_decode_attention: returns out bf16 [B, Hq, 128]."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = Workspace(B, Hq, Hkv, Lmax, n_splits, device=q.device)
+    dims = dims_of(B, Hq, Hkv, Lmax, d)
+    k0p = _dev(k0, "k0", torch.bfloat16) if k0 is not None else None
+    st = load().sr_decode_attention(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+        _dev(v_cache, "v_cache", torch.bfloat16), k0p, _dev(v0, "v0", torch.bfloat16),
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(active_list, "active_list", torch.int32),
+        int(n_splits), _dev(out, "out", torch.bfloat16), ctypes.c_void_p(workspace.ptr), workspace.nbytes,
+        _stream(stream))
+    _check("sr_decode_attention", st)
+    return out
+
+
+def grid_size() -> int:
+    return int(load().sr_decode_grid_size())
+
+
+class Decoder:
+    """Owns the route buffers and the workspace for repeated decode steps of
+    one layer shape: step() = sr_route then sr_decode_attention, both async on
+    the current stream."""
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, max_seq_len, max_splits: int = 0, device="cuda"):
+        self.shape = (batch, n_q_heads, n_kv_heads, max_seq_len)
+        U = batch * n_kv_heads
+        self.route_mask = torch.empty(U, dtype=torch.uint8, device=device)
+        self.active_list = torch.empty(1 + U, dtype=torch.int32, device=device)
+        self.out = torch.empty(batch, n_q_heads, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.workspace = Workspace(batch, n_q_heads, n_kv_heads, max_seq_len, max_splits, device=device)
+
+    def step(self, q, k_cache, v_cache, k0, v0, seq_lens, tau, n_splits: int = 0, stream=None):
+        route(q, k0, tau, self.route_mask, self.active_list, stream)
+        decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, self.active_list, self.out, n_splits,
+                         self.workspace, stream)
+        return self.out

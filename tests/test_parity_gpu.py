@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded bf16 inputs. Masks and active lists bit-exact; sink outputs equal
+v0 bit for bit; active outputs within the tolerances of tests/gpu_helpers.py."""
+import pytest
+import torch
+
+import oracle
+from kv_cache_routing_sr_b200 import inputs, native
+from tests import gpu_helpers as H
+from tests.conftest import cuda_available
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+FULL = ["tiny_4k", "llama8b_128k", "llama8b_512k", "llama70b_ragged", "llava7b_mha"]
+
+
+# ---- routing ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", FULL)
+def test_route_bit_exact_full_size(name):
+    x = inputs.make(name, seed=0, device=DEV)
+    mask_g, act_g = native.route(x.q, x.k0, x.tau)
+    torch.cuda.synchronize()
+    mask_r, act_r, score = oracle.route(x.q.cpu(), x.k0.cpu(), H.tau32(x.tau))
+    H.assert_route_equal(mask_g.cpu(), act_g.cpu(), mask_r, act_r)
+    assert (score - x.tau).abs().min().item() >= 0.05
+    assert torch.equal(mask_r, x.planted_sink.flatten().to(torch.uint8))
+
+
+def test_route_mixed_heads_use_the_minimum():
+    """A group with one non-sink head is active; ties at tau route."""
+    x = inputs.make("tiny_4k", seed=1, device=DEV, max_ctx=64)
+    q = x.q.clone()
+    q[0, 1] = x.q[0, 16]  # group 0 (sink) gets one head from an active group
+    m, a = native.route(q, x.k0, x.tau)
+    mr, ar, _ = oracle.route(q.cpu(), x.k0.cpu(), H.tau32(x.tau))
+    H.assert_route_equal(m.cpu(), a.cpu(), mr, ar)
+    assert int(m[0]) == 0 and int(m[1]) == 1
+
+
+def test_route_extreme_thresholds():
+    x = inputs.make("llava7b_mha", seed=2, device=DEV, max_ctx=64)
+    m, a = native.route(x.q, x.k0, float("inf"))
+    assert int(m.sum()) == 0 and int(a[0]) == 256
+    assert torch.equal(a[1:].cpu(), torch.arange(256, dtype=torch.int32))
+    m, a = native.route(x.q, x.k0, float("-inf"))
+    assert int(m.sum()) == 256 and int(a[0]) == 0
+
+
+# ---- attention, whole problem compared at reduced contexts --------------------------------
+
+SMALL = [
+    ("tiny_4k", {}),
+    ("llama8b_128k", dict(max_ctx=3000)),
+    ("llama8b_512k", dict(max_ctx=2048, sink_fraction=0.25)),
+    ("llama70b_ragged", dict(max_ctx=2500, poison_padding=True)),
+    ("llava7b_mha", dict(max_ctx=1500, batch=3)),
+]
+
+
+@pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] for s in SMALL])
+def test_decode_matches_oracle_small(name, kw):
+    x = inputs.make(name, seed=11, device=DEV, **kw)
+    mask_g, act_g, out_g, _ = H.gpu_step(x)
+    ref = H.oracle_full(x, x.tau)
+    H.assert_route_equal(mask_g, act_g, ref.mask, ref.active_list)
+    M = x.n_q_heads // x.n_kv_heads
+    for u in range(x.batch * x.n_kv_heads):
+        b, g = divmod(u, x.n_kv_heads)
+        if mask_g[u]:
+            H.assert_sink_exact(out_g[b, g * M:(g + 1) * M], x.v0[b, g])
+    act = mask_g.view(x.batch, x.n_kv_heads).repeat_interleave(M, dim=1) == 0
+    H.assert_active_close(out_g[act], ref.out[act], name)
+
+
+@pytest.mark.parametrize("n_splits", [1, 2, 7, 64, 0])
+def test_split_count_sweep(n_splits):
+    x = inputs.make("llama70b_ragged", seed=12, device=DEV, max_ctx=4096, poison_padding=True)
+    mask_g, _, out_g, _ = H.gpu_step(x, n_splits=n_splits)
+    H.check_against_oracle(x, out_g, mask_g, what=f"n_splits={n_splits}")
+
+
+@pytest.mark.parametrize("L", [1, 2, 15, 63, 64, 65, 129, 257, 4097])
+def test_ragged_lengths(L):
+    """Lengths around tile and split edges, poisoned padding behind them."""
+    x = inputs.make("tiny_4k", seed=13, device=DEV, max_ctx=4160, sink_groups=(1, 6))
+    x.seq_lens.fill_(L)
+    x.k_cache[:, :, L:] = float("nan")
+    x.v_cache[:, :, L:] = float("nan")
+    for ns in (0, 3):
+        mask_g, _, out_g, _ = H.gpu_step(x, n_splits=ns)
+        H.check_against_oracle(x, out_g, mask_g, what=f"L={L} n_splits={ns}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_group_sizes(M):
+    from tests.pins import _rand_case
+    q, k, v, k0, v0, seq = _rand_case(14 + M, 2, 3, M, 777, Lmax=800)
+    seq[1] = 555
+    x = inputs.DecodeInputs(inputs.WORKLOADS["tiny_4k"], 0, q, k, v, k0, v0, seq,
+                            torch.zeros(2, 3, dtype=torch.bool), 0.6).to(DEV)
+    for tau in (float("inf"), 0.0):
+        mask_g, _, out_g, _ = H.gpu_step(x, tau=tau)
+        mr, _, _ = oracle.route(q, k0, H.tau32(tau))
+        assert torch.equal(mask_g, mr)
+        H.check_against_oracle(x, out_g, mask_g, what=f"M={M} tau={tau}")
+
+
+# ---- full-size configs: sampled units -------------------------------------------------------
+
+def _sample(mask, k_active=2):
+    act = [u for u in range(len(mask)) if mask[u] == 0]
+    pick = act[:1] + act[-1:] if len(act) > 1 else act
+    return sorted(set(pick[:k_active] + [u for u in range(len(mask)) if mask[u]]))
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_decode_full_size_sampled(name):
+    x = inputs.make(name, seed=0, device=DEV)
+    mask_g, act_g, out_g, _ = H.gpu_step(x)
+    mask_r, act_r, _ = oracle.route(x.q.cpu(), x.k0.cpu(), H.tau32(x.tau))
+    H.assert_route_equal(mask_g, act_g, mask_r, act_r)
+    H.check_against_oracle(x, out_g, mask_g, units=_sample(mask_g), what=name)
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_512k_sink_sweep_sampled(frac):
+    x = inputs.make("llama8b_512k", seed=3, device=DEV, sink_fraction=frac)
+    mask_g, act_g, out_g, _ = H.gpu_step(x)
+    assert int(mask_g.sum()) == round(8 * frac)
+    act = [u for u in range(8) if mask_g[u] == 0]
+    H.check_against_oracle(x, out_g, mask_g, units=sorted(set(act[:1] + [u for u in range(8) if mask_g[u]])),
+                           what=f"512k frac={frac}")
+
+
+# ---- invariants, edge cases, error reporting ----------------------------------------------
+
+def test_all_sink_and_all_active():
+    x = inputs.make("llama70b_ragged", seed=15, device=DEV, max_ctx=1024)
+    mask_g, act_g, out_g, _ = H.gpu_step(x, tau=float("-inf"))
+    assert int(act_g[0]) == 0
+    M = 8
+    for u in range(32):
+        b, g = divmod(u, 8)
+        H.assert_sink_exact(out_g[b, g * M:(g + 1) * M], x.v0[b, g])
+    mask_g, act_g, out_g, _ = H.gpu_step(x, tau=float("inf"))
+    assert int(act_g[0]) == 32
+    H.check_against_oracle(x, out_g, mask_g)
+
+
+def test_single_unit():
+    x = inputs.make("llama8b_128k", seed=16, device=DEV, max_ctx=5000, batch=1)
+    x = inputs.DecodeInputs(x.workload, 0, x.q[:, :4].contiguous(), x.k_cache[:, :1].contiguous(),
+                            x.v_cache[:, :1].contiguous(), x.k0[:, :1].contiguous(), x.v0[:, :1].contiguous(),
+                            x.seq_lens, x.planted_sink[:, :1], 0.6)
+    for tau in (float("inf"), float("-inf")):
+        mask_g, _, out_g, _ = H.gpu_step(x, tau=tau)
+        H.check_against_oracle(x, out_g, mask_g)
+
+
+def test_routing_isolation_on_gpu():
+    x = inputs.make("llama8b_128k", seed=17, device=DEV, max_ctx=8192)
+    mask_r, _, out_r, _ = H.gpu_step(x)
+    _, _, out_d, _ = H.gpu_step(x, tau=float("inf"))
+    act = mask_r.view(1, 8).repeat_interleave(4, dim=1) == 0
+    mx, _, _ = H.active_error(out_r[act], out_d[act].double())
+    assert mx <= 2 ** -8 * out_d[act].double().abs().max().item() + 1e-6
+
+
+def test_repeat_calls_identical_and_counters_reset():
+    x = inputs.make("llama70b_ragged", seed=18, device=DEV, max_ctx=3000)
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    outs = []
+    for _ in range(3):
+        _, _, o, _ = H.gpu_step(x, decoder=dec)
+        outs.append(o.clone())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    U = x.batch * x.n_kv_heads
+    cnt = dec.workspace.view[256:256 + 4 * U].view(torch.int32)
+    assert int(cnt.abs().sum()) == 0
+    assert dec.workspace.device_error() == 0
+
+
+def test_seq_len_out_of_range_is_clamped_and_reported():
+    x = inputs.make("tiny_4k", seed=19, device=DEV, max_ctx=512)
+    ref_hi = inputs.DecodeInputs(x.workload, 0, x.q, x.k_cache, x.v_cache, x.k0, x.v0,
+                                 torch.full((1,), 512, dtype=torch.int32, device=DEV), x.planted_sink, x.tau)
+    x.seq_lens.fill_(10_000)
+    dec = native.Decoder(1, 32, 8, 512)
+    mask_g, _, out_g, _ = H.gpu_step(x, decoder=dec)
+    assert dec.workspace.device_error() & native.SR_DEVERR_SEQ_LEN
+    H.check_against_oracle(ref_hi, out_g, mask_g)
+    dec.workspace.clear_device_error()
+    assert dec.workspace.device_error() == 0
+
+
+def test_bad_active_list_is_reported_not_fatal():
+    x = inputs.make("tiny_4k", seed=20, device=DEV, max_ctx=256)
+    dec = native.Decoder(1, 32, 8, 256)
+    bad = torch.tensor([3, 5, 4, 6, 0, 0, 0, 0, 0], dtype=torch.int32, device=DEV)  # 4 after 5: out of order
+    native.decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, bad, dec.out,
+                            workspace=dec.workspace)
+    torch.cuda.synchronize()
+    assert dec.workspace.device_error() & native.SR_DEVERR_ACTIVE_LIST
+    assert torch.isfinite(dec.out.float()).all()
