@@ -63,6 +63,8 @@ constexpr long long kMinChunk = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull; // 2 s: far above any legitimate wait
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
+constexpr int kMergeThreads = 32 * kCWarps;
+constexpr int kMergeBatch = 16; // partials in flight per thread in the final merge
 
 struct alignas(16) TileHdr {
     int32_t unit;       // flat unit b*Hkv+g
@@ -75,6 +77,9 @@ struct alignas(16) TileHdr {
     int32_t pad;
 };
 
+constexpr int kUnitCache = 8; // active entries the producer gets from the prologue
+constexpr int kSeqTab = 4096;  // seq_lens entries staged in shared memory
+
 struct Misc {
     int abort_flag;
     int is_last;
@@ -82,6 +87,8 @@ struct Misc {
     int pad;
     long long s0;
     long long wsum[kCWarps + 1];
+    int cache_u[kUnitCache];
+    int cache_l[kUnitCache];
 };
 
 struct Params {
@@ -108,10 +115,13 @@ template <int RB, int STAGES> struct Cfg {
     static constexpr int OFF_HDR = OFF_ML + kCWarps * kMaxGroup * 8;
     static constexpr int OFF_BAR = OFF_HDR + STAGES * (int)sizeof(TileHdr);
     static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
-    static constexpr int OFF_BITMAP = OFF_MISC + 128;
+    static constexpr int OFF_BITMAP = OFF_MISC + 256;
     static constexpr int BYTES = OFF_BITMAP + SR_MAX_UNITS / 8;
     static constexpr int ALLOC = BYTES + 1024; // room to align the base to 1024 B
-    static_assert(sizeof(Misc) <= 128, "misc block");
+    static_assert(sizeof(Misc) <= 256, "misc block");
+    // Prologue tables (seq_lens, active lengths, active units) live in the
+    // stage buffers before the first copy is issued.
+    static_assert(kSeqTab * 4 + SR_MAX_UNITS * 6 <= STAGES * STAGE, "prologue tables");
     static_assert(BN <= 256, "TMA box rows");
     static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
 };
@@ -213,8 +223,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         misc->i0 = INT_MAX;
         misc->s0 = 0;
     }
+    if (warp == kCWarps && lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
     for (int w = tid; w < (U + 31) / 32; w += kThreads)
         bitmap[w] = 0;
+    int32_t *seqtab = reinterpret_cast<int32_t *>(smem);
+    int32_t *ltab = seqtab + kSeqTab;
+    int16_t *utab = reinterpret_cast<int16_t *>(ltab + SR_MAX_UNITS);
+    const bool seq_smem = p.B <= kSeqTab;
+    // seq_lens is a caller input that was complete before the routing kernel
+    // ran, so it is staged before the dependency wait; the active list is the
+    // routing kernel's output and is read only after it.
+    if (seq_smem)
+        for (int b = tid; b < p.B; b += kThreads)
+            seqtab[b] = __ldg(p.seq_lens + b);
+    grid_dependency_wait();
+    grid_launch_dependents();
     __syncthreads();
 
     int errbits = 0;
@@ -224,13 +250,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         n = n < 0 ? 0 : U;
     }
     long long local = 0;
-    for (int i = tid; i < n; i += kThreads) {
-        int u;
-        const int L = active_len(p, i, U, u, errbits);
-        if (L > 0) {
+    for (int i = tid; i < U; i += kThreads) {
+        const int u = __ldg(p.active + 1 + i);
+        const int prev = (i > 0) ? __ldg(p.active + i) : -1;
+        if (i >= n)
+            continue;
+        int L = 0;
+        if (u < 0 || u >= U || u <= prev) {
+            errbits |= SR_DEVERR_ACTIVE_LIST;
+        } else {
+            L = seq_smem ? seqtab[u / p.Hkv] : __ldg(p.seq_lens + u / p.Hkv);
+            if (L < 1 || L > p.Lmax) {
+                errbits |= SR_DEVERR_SEQ_LEN;
+                L = L < 1 ? 1 : p.Lmax;
+            }
             atomicOr(&bitmap[u >> 5], 1u << (u & 31));
-            local += L;
         }
+        ltab[i] = L;
+        utab[i] = (int16_t)(L > 0 ? u : -1);
+        local += L;
     }
     long long P;
     (void)block_scan(local, misc, &P);
@@ -249,9 +287,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             long long carry = 0;
             for (int base = 0; base < n; base += kThreads) {
                 const int i = base + tid;
-                int L = 0, u, dummy = 0;
-                if (i < n)
-                    L = active_len(p, i, U, u, dummy);
+                const int L = (i < n) ? ltab[i] : 0;
                 long long tot;
                 const long long incl = block_scan(L, misc, &tot);
                 const long long S = carry + incl - L;
@@ -264,13 +300,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         }
     }
     __syncthreads();
+    if (tid < kUnitCache && misc->i0 < n) {
+        const int i = misc->i0 + tid;
+        misc->cache_u[tid] = (i < n) ? (int)utab[i] : -1;
+        misc->cache_l[tid] = (i < n) ? ltab[i] : 0;
+    }
+    __syncthreads(); // the stage buffers are free for the copies from here on
 
     // ---------------------------------------------------------------- producer
     if (warp == kCWarps) {
         if (lane != 0)
             return;
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
         const uint64_t pol = l2_policy_evict_first();
         int stage = 0;
         uint32_t ph = 0;
@@ -333,11 +373,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 
         if (p.n_splits == 0) {
             if (P > 0 && r0 < P) {
-                int i = misc->i0;
+                const int i0 = misc->i0;
+                int i = i0;
                 long long S = misc->s0;
                 while (ok && i < n && S < r1) {
-                    int u, dummy = 0;
-                    const int L = active_len(p, i, U, u, dummy);
+                    int u, L;
+                    if (i - i0 < kUnitCache) {
+                        u = misc->cache_u[i - i0];
+                        L = misc->cache_l[i - i0];
+                    } else {
+                        int dummy = 0;
+                        L = active_len(p, i, U, u, dummy);
+                    }
                     if (L > 0) {
                         const long long b0 = (r0 > S ? r0 : S) - S;
                         const long long e0 = (r1 < S + L ? r1 : S + L) - S;
@@ -442,11 +489,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             break;
         const uint32_t st = sbase + stage * C::STAGE;
         if (h.flags & kFirst) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-            mrun[0] = mrun[1] = -INFINITY;
-            lrun[0] = lrun[1] = 0.f;
+            // (m, l, O) are at their initial values here: the kernel starts
+            // with them and every split's last tile resets them.
             if (h.nvalid > 0) {
                 const uint32_t *qs = reinterpret_cast<const uint32_t *>(smem + C::OFF_Q + stage * C::QBYTES);
 #pragma unroll
@@ -626,6 +670,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 __stcg(p.part_ml + (size_t)h.slot * M + ctid, make_float2(Mh, Lh));
             }
             __threadfence();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+            mrun[0] = mrun[1] = -INFINITY;
+            lrun[0] = lrun[1] = 0.f;
             if (!(ok = cbar_sync()))
                 break;
             if (ctid == 0)
@@ -633,37 +682,96 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             if (!(ok = cbar_sync()))
                 break;
             if (misc->is_last) {
-                // ---- last split of the unit to finish: merge all its partials
+                // ---- last split of the unit to finish: merge all its partials.
+                // Threads own float4 columns of the unit's [M x 128] output;
+                // when M < 4 the threads also split the partials into groups.
+                // Each thread keeps kMergeBatch partials in flight; the merge
+                // order is fixed, so the result does not depend on which CTA
+                // finished last.
                 __threadfence();
                 const int b = h.unit / p.Hkv, gg = h.unit - b * p.Hkv;
-                for (int idx = ctid; idx < M * 32; idx += 32 * kCWarps) {
-                    const int head = idx >> 5, d4 = (idx & 31) * 4;
+                const int ncol = M * 32;
+                const int cpg = ncol < kMergeThreads ? ncol : kMergeThreads;
+                const int sgrp = kMergeThreads / cpg;
+                const int grp = ctid / cpg;
+                for (int col = ctid % cpg; col < ncol; col += cpg) {
+                    const int head = col >> 5, d4 = (col & 31) * 4;
                     float m = -INFINITY, l = 0.f;
                     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int j = 0; j < h.nseg; ++j) {
-                        const size_t sl = (size_t)(h.slot_first + j) * M + head;
-                        const float2 x = __ldcg(p.part_ml + sl);
-                        const float4 y = __ldcg(reinterpret_cast<const float4 *>(p.part_o + sl * kHeadDim + d4));
-                        if (x.x == -INFINITY)
-                            continue;
-                        const float mn = fmaxf(m, x.x);
-                        const float a = exp2f(m - mn), c = exp2f(x.x - mn);
-                        l = l * a + x.y * c;
-                        acc.x = acc.x * a + y.x * c;
-                        acc.y = acc.y * a + y.y * c;
-                        acc.z = acc.z * a + y.z * c;
-                        acc.w = acc.w * a + y.w * c;
-                        m = mn;
+                    for (int j0 = grp; j0 < h.nseg; j0 += sgrp * kMergeBatch) {
+                        float2 x[kMergeBatch];
+                        float4 y[kMergeBatch];
+#pragma unroll
+                        for (int k = 0; k < kMergeBatch; ++k) {
+                            const int j = j0 + k * sgrp;
+                            if (j < h.nseg) {
+                                const size_t sl = (size_t)(h.slot_first + j) * M + head;
+                                x[k] = __ldcg(p.part_ml + sl);
+                                y[k] = __ldcg(reinterpret_cast<const float4 *>(p.part_o + sl * kHeadDim + d4));
+                            } else {
+                                x[k] = make_float2(-INFINITY, 0.f);
+                                y[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < kMergeBatch; ++k) {
+                            if (x[k].x == -INFINITY)
+                                continue; // empty split
+                            const float mn = fmaxf(m, x[k].x);
+                            const float a = exp2f(m - mn), c = exp2f(x[k].x - mn);
+                            l = l * a + x[k].y * c;
+                            acc.x = acc.x * a + y[k].x * c;
+                            acc.y = acc.y * a + y[k].y * c;
+                            acc.z = acc.z * a + y[k].z * c;
+                            acc.w = acc.w * a + y[k].w * c;
+                            m = mn;
+                        }
                     }
-                    const float inv = 1.f / l;
-                    uint2 packed;
-                    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-                    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-                    *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim + d4) =
-                        packed;
+                    if (sgrp == 1) {
+                        const float inv = 1.f / l;
+                        uint2 packed;
+                        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+                        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+                        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim +
+                                                   d4) = packed;
+                    } else {
+                        *reinterpret_cast<float4 *>(comb + 4 * ctid) = acc;
+                        *reinterpret_cast<float2 *>(comb + 4 * kMergeThreads + 2 * ctid) = make_float2(m, l);
+                    }
+                }
+                if (sgrp > 1) {
+                    if (!(ok = cbar_sync()))
+                        break;
+                    if (ctid < cpg) {
+                        const int head = ctid >> 5, d4 = (ctid & 31) * 4;
+                        float m = -INFINITY;
+                        for (int q = 0; q < sgrp; ++q)
+                            m = fmaxf(m, comb[4 * kMergeThreads + 2 * (q * cpg + ctid)]);
+                        float l = 0.f;
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int q = 0; q < sgrp; ++q) {
+                            const int e = q * cpg + ctid;
+                            const float2 ml = *reinterpret_cast<const float2 *>(comb + 4 * kMergeThreads + 2 * e);
+                            if (ml.x == -INFINITY)
+                                continue;
+                            const float c = exp2f(ml.x - m);
+                            const float4 y = *reinterpret_cast<const float4 *>(comb + 4 * e);
+                            l += ml.y * c;
+                            acc.x += y.x * c, acc.y += y.y * c, acc.z += y.z * c, acc.w += y.w * c;
+                        }
+                        const float inv = 1.f / l;
+                        uint2 packed;
+                        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+                        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+                        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim +
+                                                   d4) = packed;
+                    }
                 }
                 if (ctid == 0)
                     p.cnt[h.unit] = 0;
+                // Shared scratch (comb, mlsm) is reused by the next split's end.
+                if (!(ok = cbar_sync()))
+                    break;
             }
         }
         if (++stage == STAGES) {
@@ -798,8 +906,18 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
     p.M = a.n_q_heads / a.n_kv_heads;
     p.Lmax = a.max_seq_len;
     p.n_splits = a.n_splits;
-    decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES><<<info->grid, kThreads, DecodeCfg::ALLOC, stream>>>(tmK, tmV, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(info->grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = DecodeCfg::ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES>, tmK, tmV, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 } // namespace sr

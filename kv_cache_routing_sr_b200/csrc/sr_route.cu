@@ -10,20 +10,21 @@
 //
 // Layout: one CTA of 32 warps. Each warp owns whole units (b, g): lane l holds
 // elements 4l..4l+3 of k0_g and of each query head, so a unit's dot products
-// and squared norms are warp shuffle reductions in fp32. The compaction writes
+// and squared norms are warp shuffle reductions in fp32. All loads of a pass
+// are issued before the first reduction (one memory round trip per pass). The compaction writes
 // active units in ascending order with warp ballots and a block prefix, so no
 // CTA of the decode kernel is ever bound to a sink unit.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "sr_internal.h"
+#include "sr_ptx.cuh"
 
 namespace sr {
 namespace {
 
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kUnroll = 4; // units in flight per warp
 
 __device__ __forceinline__ float warp_sum(float x)
 {
@@ -33,69 +34,78 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
-__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4])
+__device__ __forceinline__ void widen4(uint2 raw, float (&v)[4])
 {
-    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
     v[0] = fa.x, v[1] = fa.y, v[2] = fb.x, v[3] = fb.y;
 }
 
+__device__ __forceinline__ float dot4(const float (&a)[4], const float (&b)[4])
+{
+    return a[0] * b[0] + a[1] * b[1] + a[2] * b[2] + a[3] * b[3];
+}
+
+// M = query heads per KV head (compile time). Each warp routes UNR units per
+// pass, with every load of those units (k0 and the M query heads) issued before
+// the first reduction, so a pass costs one memory round trip.
+template <int M>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k0, float tau,
-             uint8_t *__restrict__ mask, int32_t *__restrict__ active, int B, int Hq, int Hkv)
+             uint8_t *__restrict__ mask, int32_t *__restrict__ active, int B, int Hkv)
 {
+    constexpr int UNR = (8 / M) > 0 ? (8 / M) : 1;
     extern __shared__ uint8_t sink_flag[]; // [B*Hkv]
     __shared__ int32_t warp_cnt[kRouteWarps];
     __shared__ int32_t warp_off[kRouteWarps + 1];
 
+    // Inputs may come from the previous kernel in the stream, and the previous
+    // decode step may still read route_mask / active_list: wait for it, then
+    // let the decode kernel that follows launch and run its prologue.
+    grid_dependency_wait();
+    grid_launch_dependents();
+
     const int U = B * Hkv;
-    const int M = Hq / Hkv;
+    const int Hq = Hkv * M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    for (int base = warp; base < U; base += kRouteWarps * kUnroll) {
-        float s[kUnroll];
+    for (int base = warp; base < U; base += kRouteWarps * UNR) {
+        uint2 kraw[UNR], qraw[UNR][M];
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k)
-            s[k] = INFINITY;
-        float kv[kUnroll][4] = {};
-#pragma unroll
-        for (int k = 0; k < kUnroll; ++k) {
+        for (int k = 0; k < UNR; ++k) {
             const int u = base + k * kRouteWarps;
-            if (u < U)
-                load4(k0 + (size_t)u * kHeadDim + 4 * lane, kv[k]);
-        }
-        float kk[kUnroll];
+            kraw[k] = make_uint2(0u, 0u);
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k)
-            kk[k] = warp_sum(kv[k][0] * kv[k][0] + kv[k][1] * kv[k][1] + kv[k][2] * kv[k][2] + kv[k][3] * kv[k][3]);
-        for (int m = 0; m < M; ++m) {
-            float qv[kUnroll][4] = {};
+            for (int m = 0; m < M; ++m)
+                qraw[k][m] = make_uint2(0u, 0u);
+            if (u < U) {
+                const int b = u / Hkv, g = u - b * Hkv;
+                kraw[k] = *reinterpret_cast<const uint2 *>(k0 + (size_t)u * kHeadDim + 4 * lane);
 #pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
-                const int u = base + k * kRouteWarps;
-                if (u < U) {
-                    const int b = u / Hkv, g = u - b * Hkv;
-                    load4(q + ((size_t)b * Hq + (size_t)g * M + m) * kHeadDim + 4 * lane, qv[k]);
-                }
+                for (int m = 0; m < M; ++m)
+                    qraw[k][m] = *reinterpret_cast<const uint2 *>(
+                        q + ((size_t)b * Hq + (size_t)g * M + m) * kHeadDim + 4 * lane);
             }
+        }
 #pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
-                const float dot = warp_sum(qv[k][0] * kv[k][0] + qv[k][1] * kv[k][1] + qv[k][2] * kv[k][2] +
-                                           qv[k][3] * kv[k][3]);
-                const float qq =
-                    warp_sum(qv[k][0] * qv[k][0] + qv[k][1] * qv[k][1] + qv[k][2] * qv[k][2] + qv[k][3] * qv[k][3]);
-                const float c = (qq == 0.f || kk[k] == 0.f) ? 0.f : dot / (sqrtf(qq) * sqrtf(kk[k]));
+        for (int k = 0; k < UNR; ++k) {
+            const int u = base + k * kRouteWarps;
+            float kv[4];
+            widen4(kraw[k], kv);
+            const float kk = warp_sum(dot4(kv, kv));
+            float s = INFINITY;
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                float qv[4];
+                widen4(qraw[k][m], qv);
+                const float dot = warp_sum(dot4(qv, kv));
+                const float qq = warp_sum(dot4(qv, qv));
+                const float c = (qq == 0.f || kk == 0.f) ? 0.f : dot / (sqrtf(qq) * sqrtf(kk));
                 // A NaN cosine never lowers the minimum (same rule as a "<" scan).
-                s[k] = (c < s[k]) ? c : s[k];
+                s = (c < s) ? c : s;
             }
-        }
-#pragma unroll
-        for (int k = 0; k < kUnroll; ++k) {
-            const int u = base + k * kRouteWarps;
             if (u < U && lane == 0) {
-                const uint8_t sink = (s[k] >= tau) ? 1 : 0;
+                const uint8_t sink = (s >= tau) ? 1 : 0;
                 mask[u] = sink;
                 sink_flag[u] = sink;
             }
@@ -136,15 +146,46 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
         active[0] = total;
 }
 
+template <int M>
+cudaError_t launch_route_m(const RouteArgs &a, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = (size_t)a.batch * a.n_kv_heads;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, route_kernel<M>, static_cast<const __nv_bfloat16 *>(a.q),
+                              static_cast<const __nv_bfloat16 *>(a.k0), a.tau, a.mask, a.active, a.batch,
+                              a.n_kv_heads);
+}
+
 } // namespace
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream)
 {
-    const int U = a.batch * a.n_kv_heads;
-    route_kernel<<<1, kRouteThreads, (size_t)U, stream>>>(
-        static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k0), a.tau, a.mask, a.active,
-        a.batch, a.n_q_heads, a.n_kv_heads);
-    return cudaGetLastError();
+    cudaError_t e;
+    switch (a.n_q_heads / a.n_kv_heads) {
+    case 1:
+        e = launch_route_m<1>(a, stream);
+        break;
+    case 2:
+        e = launch_route_m<2>(a, stream);
+        break;
+    case 4:
+        e = launch_route_m<4>(a, stream);
+        break;
+    case 8:
+        e = launch_route_m<8>(a, stream);
+        break;
+    default:
+        return cudaErrorInvalidValue;
+    }
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 } // namespace sr
