@@ -713,17 +713,26 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                                 y[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                             }
                         }
+                        // One rescale per batch: the batch maximum first,
+                        // then independent weights (empty splits weigh 0).
+                        float mb = -INFINITY;
 #pragma unroll
-                        for (int k = 0; k < kMergeBatch; ++k) {
-                            if (x[k].x == -INFINITY)
-                                continue; // empty split
-                            const float mn = fmaxf(m, x[k].x);
-                            const float a = exp2f(m - mn), c = exp2f(x[k].x - mn);
-                            l = l * a + x[k].y * c;
-                            acc.x = acc.x * a + y[k].x * c;
-                            acc.y = acc.y * a + y[k].y * c;
-                            acc.z = acc.z * a + y[k].z * c;
-                            acc.w = acc.w * a + y[k].w * c;
+                        for (int k = 0; k < kMergeBatch; ++k)
+                            mb = fmaxf(mb, x[k].x);
+                        const float mn = fmaxf(m, mb);
+                        if (mn != -INFINITY) {
+                            const float a = exp2f(m - mn);
+                            l *= a;
+                            acc.x *= a, acc.y *= a, acc.z *= a, acc.w *= a;
+#pragma unroll
+                            for (int k = 0; k < kMergeBatch; ++k) {
+                                const float c = exp2f(x[k].x - mn);
+                                l += x[k].y * c;
+                                acc.x += y[k].x * c;
+                                acc.y += y[k].y * c;
+                                acc.z += y[k].z * c;
+                                acc.w += y[k].w * c;
+                            }
                             m = mn;
                         }
                     }
