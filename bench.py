@@ -101,6 +101,26 @@ def dist_env():
     return world, rank, local
 
 
+def reduce_max(value: float, device, world: int) -> float:
+    """Max of a per-rank float over all ranks (identity with one rank). The
+    device is the process group's: a CUDA device for NCCL, the CPU for gloo."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_us(max_total_ms: float, steps: int, world: int) -> tuple[float, float]:
+    """(slowest rank's µs per layer-step, whole-job µs per layer-step): every rank
+    runs `steps` independent layer-steps, so the job completes world*steps of
+    them in the slowest rank's time."""
+    per_rank = max_total_ms * 1e3 / steps
+    return per_rank, per_rank / world
+
+
 def active_units_of(active_list_cpu):
     n = int(active_list_cpu[0])
     return [int(u) for u in active_list_cpu[1:1 + n]]
@@ -330,14 +350,12 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dev, world)
 
     peak, peak_kind = hbm_peak()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    # fp32 so that torch sums it in place (a pure 256 MiB read; integer sums would
+    # first widen the buffer with a 2 GB write).
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     x = inputs.make(args.config, seed=args.seed + 1000 * rank, device=dev)
     clocks = ClockSampler(local)
     clocks.start()
@@ -349,8 +367,7 @@ def run_ours(args):
     K = args.steps
     sum_ms = max_over_ranks(sum(r["tot"]))
     sum_ms_dis = max_over_ranks(sum(r["tot_disabled"]))
-    us_step = sum_ms * 1e3 / K  # slowest rank's µs per layer-step
-    value = sum_ms * 1e3 / (K * world)  # whole job: time / all layer-steps of all ranks
+    us_step, value = aggregate_us(sum_ms, K, world)
     dec_us = statistics.mean(r["decode"]) * 1e3
     route_us = statistics.median(r["route"]) * 1e3
     eff_gbs = r["need"] / (us_step * 1e-6) / 1e9
