@@ -168,6 +168,47 @@ int32_t sr_decode_grid_size(void);
 /* Message of the last CUDA error seen by this library on this thread ("" if none). */
 const char *sr_last_cuda_error(void);
 
+/* Size of the fixed scratch array behind sr_decode_attention_static_scratch. */
+#define SR_STATIC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * sr_decode_attention_static_scratch -- sr_decode_attention without a
+ * workspace argument, for callers that cannot allocate device memory. (An
+ * engineering addition: the paper and its code have no counterpart.)
+ *
+ * Who needs it: code that only ever receives its input and output buffers and
+ * may not call cudaMalloc -- a plugin whose host framework owns every device
+ * allocation and passes no scratch buffer through its fixed interface, a
+ * serving runtime that plans all memory at start-up and forbids allocation on
+ * the decode path (cudaMalloc can synchronise the device and fragment a
+ * pre-planned pool), or a certified deployment that bans dynamic allocation
+ * after initialisation.
+ *
+ * The decode kernel's scratch (error word, per-unit counters, split partials)
+ * is a fixed array of SR_STATIC_SCRATCH_BYTES compiled into this library; every
+ * GPU that loads the library holds it until the process exits. Arguments,
+ * results and errors are those of sr_decode_attention, with these differences:
+ *   - no workspace: dims and n_splits whose scratch would exceed
+ *     SR_STATIC_SCRATCH_BYTES are rejected with SR_ERR_WORKSPACE (at n_splits =
+ *     0 this admits B*Hkv up to about 990 with M = 8, 3000 with M = 4, 15000
+ *     with M = 1);
+ *   - device_error: optional device pointer (NULL = not wanted) that receives
+ *     the launch's device error word (SR_DEVERR_* bits), stream-ordered;
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) and may load the module there; make that first
+ *     call before any stream capture;
+ *   - every call on a device shares the one array: each call clears the error
+ *     word and the counters it needs, so calls in sequence on one stream are
+ *     fine, but calls that overlap on the GPU (different streams, or host
+ *     threads without ordering) race on the array and must be serialised.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+sr_status sr_decode_attention_static_scratch(const sr_dims *dims, const void *q, const void *k_cache,
+                                             const void *v_cache, const void *k0, const void *v0,
+                                             const int32_t *seq_lens, const int32_t *active_list,
+                                             int32_t n_splits, void *out, int32_t *device_error,
+                                             void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -45,6 +45,8 @@ cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
 } // namespace
 
+sr_status sr::record_cuda_failure(cudaError_t e) { return cuda_fail(e); }
+
 extern "C" {
 
 const char *sr_status_string(sr_status s)

@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "sinkrouter.h"
+
 namespace sr {
 
 constexpr int kHeadDim = 128;
@@ -62,5 +64,7 @@ cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 // Persistent CTAs of the decode kernel on the current device (0 on error).
 int decode_grid_size();
+// Records a CUDA failure for sr_last_cuda_error and returns SR_ERR_CUDA.
+sr_status record_cuda_failure(cudaError_t e);
 
 } // namespace sr

@@ -40,7 +40,7 @@ _lib = None
 
 EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_decode_attention",
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
-           "sr_last_cuda_error"]
+           "sr_last_cuda_error", "sr_decode_attention_static_scratch"]
 
 
 def load(path: str = LIBRARY):
@@ -72,6 +72,8 @@ def load(path: str = LIBRARY):
     lib.sr_decode_grid_size.restype = i32
     lib.sr_last_cuda_error.argtypes = []
     lib.sr_last_cuda_error.restype = ctypes.c_char_p
+    lib.sr_decode_attention_static_scratch.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
+    lib.sr_decode_attention_static_scratch.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -167,6 +169,28 @@ def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=Non
         int(n_splits), _dev(out, "out", torch.bfloat16), ctypes.c_void_p(workspace.ptr), workspace.nbytes,
         _stream(stream))
     _check("sr_decode_attention", st)
+    return out
+
+
+def decode_attention_static_scratch(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=None,
+                                    n_splits: int = 0, device_error=None, stream=None):
+    """sr_decode_attention_static_scratch: the decode step with the library's
+    fixed scratch array instead of a workspace (no device allocation by the
+    library). ``device_error``: optional int32 CUDA tensor of one element that
+    receives the launch's device error bits. Returns out bf16 [B, Hq, 128]."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    dims = dims_of(B, Hq, Hkv, Lmax, d)
+    k0p = _dev(k0, "k0", torch.bfloat16) if k0 is not None else None
+    errp = _dev(device_error, "device_error", torch.int32) if device_error is not None else None
+    st = load().sr_decode_attention_static_scratch(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+        _dev(v_cache, "v_cache", torch.bfloat16), k0p, _dev(v0, "v0", torch.bfloat16),
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(active_list, "active_list", torch.int32),
+        int(n_splits), _dev(out, "out", torch.bfloat16), errp, _stream(stream))
+    _check("sr_decode_attention_static_scratch", st)
     return out
 
 
