@@ -205,69 +205,93 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # our arm
 
-def time_steps(native, dec, x, tau, steps, flush, barrier):
-    """Per-step device times (ms) of `steps` layer-steps (route + decode), with
-    events only around the pair so that the decode launch can overlap the
-    routing kernel (programmatic dependent launch). L2 is flushed before each
-    step by reading a 256 MiB buffer, outside the events."""
+def _captured_steps(native, dec, x, tau, steps, flush, split_events, fused):
+    """Capture `steps` layer-steps in ONE CUDA graph, as a decode forward would
+    run them: before each step an L2 flush (a 256 MiB read), then an event and
+    the step, then an event. The step is either the single fused launch
+    (sr_route_decode_attention) or sr_route then sr_decode_attention; for the
+    latter, split_events=True puts an event between the two kernels (per-kernel
+    times), otherwise the decode launch overlaps routing through its
+    programmatic dependency."""
     import torch
-    st = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(steps):
+    # external events: recorded as timestamps by the graph's event nodes
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    args = (x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens)
+    side = torch.cuda.Stream(device=x.q.device)
+    side.wait_stream(torch.cuda.current_stream(x.q.device))
+    with torch.cuda.stream(side):  # warm-up outside the capture
+        dec.step(*args, tau)
+        dec.step_fused(*args, tau)
         flush.sum()
-        ev[i][0].record(st)
-        native.route(x.q, x.k0, tau, dec.route_mask, dec.active_list)
-        native.decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, dec.active_list, dec.out,
-                                0, dec.workspace)
-        ev[i][1].record(st)
+    torch.cuda.current_stream(x.q.device).wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = torch.cuda.current_stream()
+        for i in range(steps):
+            flush.sum()
+            ev[i][0].record(st)
+            if fused:
+                native.route_decode_attention(*args, tau, dec.out, dec.route_mask, dec.active_list, 0,
+                                              dec.workspace)
+            else:
+                native.route(x.q, x.k0, tau, dec.route_mask, dec.active_list)
+                if split_events:
+                    ev[i][1].record(st)
+                native.decode_attention(*args, dec.active_list, dec.out, 0, dec.workspace)
+            ev[i][2].record(st)
+    return g, ev
+
+
+def time_steps(native, dec, x, tau, steps, warmup, flush, barrier, fused):
+    """Per-step device times (ms): events bracket the step only."""
+    import torch
+    gw, _ = _captured_steps(native, dec, x, tau, warmup, flush, False, fused)
+    g, ev = _captured_steps(native, dec, x, tau, steps, flush, False, fused)
+    gw.replay()
+    barrier()
+    torch.cuda.synchronize()
+    g.replay()
     torch.cuda.synchronize()
     barrier()
-    return [e[0].elapsed_time(e[1]) for e in ev]
+    return [e[0].elapsed_time(e[2]) for e in ev]
 
 
 def time_kernels(native, dec, x, tau, steps, flush):
-    """Per-kernel device times (ms): events around each launch on its stream
-    (an event between the two launches also removes their overlap)."""
+    """Per-kernel device times (ms) of the two-call step with an event between
+    the two kernels (which also removes their overlap)."""
     import torch
-    st = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    torch.cuda.synchronize()
-    for i in range(steps):
-        flush.sum()
-        ev[i][0].record(st)
-        native.route(x.q, x.k0, tau, dec.route_mask, dec.active_list)
-        ev[i][1].record(st)
-        native.decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, dec.active_list, dec.out,
-                                0, dec.workspace)
-        ev[i][2].record(st)
+    g, ev = _captured_steps(native, dec, x, tau, steps, flush, True, False)
+    g.replay()
     torch.cuda.synchronize()
     return [e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev]
 
 
-def measure_workload(native, inputs, x, steps, warmup, flush, dist, barrier, peak):
-    """Routed and routing-disabled timings of one workload on this GPU."""
+def measure_workload(native, inputs, x, steps, warmup, flush, barrier, two_call=True):
+    """Timings of one workload on this GPU: the fused step (routed and with
+    routing disabled) and, if asked, the two-call step and its kernels."""
     import torch
     dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
     for _ in range(warmup):
         dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+        dec.step_fused(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
     torch.cuda.synchronize()
     err = dec.workspace.device_error()
     if err:
         raise RuntimeError(f"device error word {err} after warm-up")
     act = active_units_of(dec.active_list.cpu())
     sl = x.seq_lens.cpu().tolist()
-    need = inputs.needed_bytes(sl, act, x.n_kv_heads, x.n_q_heads, x.batch)
-    need_all = inputs.needed_bytes(sl, range(x.batch * x.n_kv_heads), x.n_kv_heads, x.n_q_heads, x.batch)
-    tot = time_steps(native, dec, x, x.tau, steps, flush, barrier)
-    rte, dms = time_kernels(native, dec, x, x.tau, steps, flush)
-    for _ in range(warmup):
-        dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, float("inf"))
-    tot_d = time_steps(native, dec, x, float("inf"), steps, flush, barrier)
-    _, dms_d = time_kernels(native, dec, x, float("inf"), steps, flush)
-    return dict(dec=dec, active=act, need=need, need_all=need_all, tot=tot, route=rte, decode=dms,
-                tot_disabled=tot_d, decode_disabled=dms_d)
+    r = dict(dec=dec, active=act, need=inputs.needed_bytes(sl, act, x.n_kv_heads, x.n_q_heads, x.batch),
+             need_all=inputs.needed_bytes(sl, range(x.batch * x.n_kv_heads), x.n_kv_heads, x.n_q_heads, x.batch))
+    r["fused"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, True)
+    r["fused_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, True)
+    if two_call:
+        r["two"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, False)
+        r["route"], r["decode"] = time_kernels(native, dec, x, x.tau, steps, flush)
+        r["two_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, False)
+    err = dec.workspace.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err} after the timed steps")
+    return r
 
 
 def e2e_measure(native, x, steps):
@@ -288,7 +312,7 @@ def e2e_measure(native, x, steps):
     def one():
         for n in names:
             dev[n].copy_(host[n], non_blocking=True)
-        dec.step(dev["q"], dev["k_cache"], dev["v_cache"], dev["k0"], dev["v0"], dev["seq_lens"], x.tau)
+        dec.step_fused(dev["q"], dev["k_cache"], dev["v_cache"], dev["k0"], dev["v0"], dev["seq_lens"], x.tau)
         out_h.copy_(dec.out, non_blocking=True)
         mask_h.copy_(dec.route_mask, non_blocking=True)
 
@@ -360,20 +384,22 @@ def run_ours(args):
     clocks = ClockSampler(local)
     clocks.start()
     t_wall = time.perf_counter()
-    r = measure_workload(native, inputs, x, args.steps, args.warmup, flush, dist, barrier, peak)
+    r = measure_workload(native, inputs, x, args.steps, args.warmup, flush, barrier)
     t_wall = time.perf_counter() - t_wall
     clk = clocks.stop()
 
     K = args.steps
-    sum_ms = max_over_ranks(sum(r["tot"]))
-    sum_ms_dis = max_over_ranks(sum(r["tot_disabled"]))
+    sum_ms = max_over_ranks(sum(r["two"]))
     us_step, value = aggregate_us(sum_ms, K, world)
+    us_dis, _ = aggregate_us(max_over_ranks(sum(r["two_disabled"])), K, world)
+    us_fused, _ = aggregate_us(max_over_ranks(sum(r["fused"])), K, world)
+    us_fused_dis, _ = aggregate_us(max_over_ranks(sum(r["fused_disabled"])), K, world)
+    step_p = [v * 1e3 for v in r["two"]]
     dec_us = statistics.mean(r["decode"]) * 1e3
     route_us = statistics.median(r["route"]) * 1e3
-    eff_gbs = r["need"] / (us_step * 1e-6) / 1e9
-    us_dis = sum_ms_dis * 1e3 / K
-    eff_gbs_dis = r["need_all"] / (us_dis * 1e-6) / 1e9
-    achieved = r["need"] / (dec_us * 1e-6) / 1e9
+    need = r["need"]
+    gbs = lambda nbytes, us: nbytes / (us * 1e-6) / 1e9  # noqa: E731
+    achieved = gbs(need, dec_us)  # the decode kernel, timed alone
     traffic = profiled_traffic()
 
     line = {
@@ -381,22 +407,29 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(us_step / 1e3, 6), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
         "config": describe_config(x, len(r["active"]), world),
-        "effective_gbs": round(eff_gbs, 1), "frac_of_hbm_peak": round(eff_gbs / peak, 4),
-        "route_us_median": round(route_us, 3), "decode_us_mean": round(dec_us, 3),
-        "step_us_p10_p50_p90": [round(statistics.quantiles(r["tot"], n=10)[i] * 1e3, 3) for i in (0, 4, 8)],
-        "needed_bytes_per_step": r["need"],
-        "routing_disabled": {"us_per_layer_step": round(us_dis, 3), "effective_gbs": round(eff_gbs_dis, 1),
-                             "frac_of_hbm_peak": round(eff_gbs_dis / peak, 4),
-                             "decode_us_mean": round(statistics.mean(r["decode_disabled"]) * 1e3, 3),
+        "path": "sr_route then sr_decode_attention (decode launch overlaps routing: programmatic dependency)",
+        "effective_gbs": round(gbs(need, us_step), 1), "frac_of_hbm_peak": round(gbs(need, us_step) / peak, 4),
+        "route_kernel_us_median": round(route_us, 3), "decode_kernel_us_mean": round(dec_us, 3),
+        "step_us_p10_p50_p90": [round(statistics.quantiles(step_p, n=10)[i], 3) for i in (0, 4, 8)],
+        "needed_bytes_per_step": need,
+        "routing_disabled": {"us_per_layer_step": round(us_dis, 3),
+                             "effective_gbs": round(gbs(r["need_all"], us_dis), 1),
+                             "frac_of_hbm_peak": round(gbs(r["need_all"], us_dis) / peak, 4),
                              "speedup_routed": round(us_dis / us_step, 3),
                              "active_fraction": round(len(r["active"]) / (x.batch * x.n_kv_heads), 4)},
+        "fused_single_launch": {"path": "sr_route_decode_attention (every CTA routes in its prologue)",
+                                "us_per_layer_step": round(us_fused, 3),
+                                "effective_gbs": round(gbs(need, us_fused), 1),
+                                "routing_disabled_us": round(us_fused_dis, 3)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "sinkrouter decode_kernel (persistent split-K scan + reduction)",
-                     "algorithmic_bytes_per_launch": r["need"], "peak_source": f"{peak_kind} HBM copy"},
+                     "kernel": "decode_kernel<1,4> (persistent split-K scan + sink copy + merge)",
+                     "algorithmic_bytes_per_launch": need, "peak_source": f"{peak_kind} HBM copy"},
         "gpu_launches": 2 * K,
-        "timing": "value/ms_per_step: events around route+decode only (launches overlap via programmatic "
-                  "dependent launch); route/decode kernel times: a second pass with an event between them",
+        "gpu_launches": K,
+        "timing": "the K timed steps are captured in one CUDA graph (per step: L2 flush read, event, the "
+                  "step, event) and replayed once; the two-call figures come from the same protocol, and its "
+                  "per-kernel times from a graph with an event between the two kernels",
         "clocks": clk,
         "timed_wall_s": round(t_wall, 3),
         "impl": "ours",
@@ -406,14 +439,13 @@ def run_ours(args):
         sweep = []
         for frac in (0.0, 0.25, 0.5, 0.75, 1.0):
             x5 = inputs.make("llama8b_512k", seed=args.seed, device=dev, sink_fraction=frac)
-            s5 = measure_workload(native, inputs, x5, max(20, min(K, 50)), args.warmup, flush, dist, barrier, peak)
-            u5 = statistics.mean(s5["tot"]) * 1e3
-            d5 = statistics.mean(s5["decode"]) * 1e3
-            ud5 = statistics.mean(s5["tot_disabled"]) * 1e3
+            s5 = measure_workload(native, inputs, x5, max(20, min(K, 50)), args.warmup, flush, barrier,
+                                  two_call=False)
+            u5 = statistics.mean(s5["fused"]) * 1e3
+            ud5 = statistics.mean(s5["fused_disabled"]) * 1e3
             sweep.append({"sink_fraction": frac, "us_per_layer_step": round(u5, 2),
                           "effective_gbs": round(s5["need"] / (u5 * 1e-6) / 1e9, 1),
-                          "decode_kernel_gbs": round(s5["need"] / (d5 * 1e-6) / 1e9, 1),
-                          "decode_frac_of_peak": round(s5["need"] / (d5 * 1e-6) / 1e9 / peak, 4),
+                          "frac_of_peak": round(s5["need"] / (u5 * 1e-6) / 1e9 / peak, 4),
                           "routing_disabled_us": round(ud5, 2), "speedup_routed": round(ud5 / u5, 3)})
             del x5, s5
             torch.cuda.empty_cache()
@@ -423,6 +455,7 @@ def run_ours(args):
         ms = max_over_ranks(ms)
         line["e2e"] = {"value": round(ms * 1e3 / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                       "path": "sr_route_decode_attention, eager launch",
                        "note": "pinned host buffers; every input (caches included) copied each step"}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         xc = x.to("cpu")

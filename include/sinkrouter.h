@@ -146,6 +146,29 @@ sr_status sr_decode_attention(const sr_dims *dims, const void *q, const void *k_
                               int32_t n_splits, void *out, void *workspace,
                               size_t workspace_bytes, void *stream);
 
+/*
+ * sr_route_decode_attention -- sr_route followed by sr_decode_attention in ONE
+ * kernel launch: every CTA of the decode kernel routes all units itself (the
+ * same fp32 arithmetic as sr_route, so the decisions are identical) and builds
+ * the work list in shared memory, which removes the routing launch and the
+ * hand-off between the two kernels from the step. Same method and passages as
+ * the two calls above; the result (route decisions and out) equals theirs bit
+ * for bit.
+ *
+ *   q, k_cache, v_cache, v0, seq_lens, n_splits, out, workspace, workspace_bytes:
+ *               as for sr_decode_attention
+ *   k0, tau     as for sr_route (k0 is required here)
+ *   route_mask  optional out uint8 [B*Hkv] (NULL = not written)
+ *   active_list optional out int32 [1 + B*Hkv] in sr_route's format (NULL = not
+ *               written); this call never reads it
+ * Errors: SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_WORKSPACE, SR_ERR_CUDA.
+ */
+sr_status sr_route_decode_attention(const sr_dims *dims, const void *q, const void *k_cache,
+                                    const void *v_cache, const void *k0, const void *v0,
+                                    const int32_t *seq_lens, float tau, int32_t n_splits,
+                                    uint8_t *route_mask, int32_t *active_list, void *out,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static description of a status code. */
 const char *sr_status_string(sr_status s);
 

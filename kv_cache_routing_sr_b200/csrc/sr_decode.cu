@@ -46,6 +46,7 @@
 #include "sinkrouter.h"
 #include "sr_internal.h"
 #include "sr_ptx.cuh"
+#include "sr_route_math.cuh"
 
 #ifndef SR_DECODE_RB
 #define SR_DECODE_RB 1 // row blocks of 16 per consumer warp and tile
@@ -77,8 +78,7 @@ struct alignas(16) TileHdr {
     int32_t pad;
 };
 
-constexpr int kUnitCache = 8; // active entries the producer gets from the prologue
-constexpr int kSeqTab = 4096;  // seq_lens entries staged in shared memory
+constexpr int kSeqTab = 4096; // seq_lens entries staged in shared memory
 
 struct Misc {
     int abort_flag;
@@ -87,8 +87,8 @@ struct Misc {
     int pad;
     long long s0;
     long long wsum[kCWarps + 1];
-    int cache_u[kUnitCache];
-    int cache_l[kUnitCache];
+    int first_bad; // first malformed entry of the active list (INT_MAX: none)
+    int first_u;   // unit of the producer's first active entry (-1: none)
 };
 
 struct Params {
@@ -102,6 +102,11 @@ struct Params {
     float *part_o;
     float2 *part_ml;
     int B, Hq, Hkv, M, Lmax, n_splits;
+    // fused routing (sr_route_decode_attention) only
+    const __nv_bfloat16 *k0;
+    float tau;
+    uint8_t *mask_out;   // may be null
+    int32_t *active_out; // may be null
 };
 
 template <int RB, int STAGES> struct Cfg {
@@ -121,7 +126,7 @@ template <int RB, int STAGES> struct Cfg {
     static_assert(sizeof(Misc) <= 256, "misc block");
     // Prologue tables (seq_lens, active lengths, active units) live in the
     // stage buffers before the first copy is issued.
-    static_assert(kSeqTab * 4 + SR_MAX_UNITS * 6 <= STAGES * STAGE, "prologue tables");
+    static_assert(kSeqTab * 4 + SR_MAX_UNITS * 7 <= STAGES * STAGE, "prologue tables");
     static_assert(BN <= 256, "TMA box rows");
     static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
 };
@@ -143,23 +148,29 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
 }
 
-// Valid length of the i-th active entry, or 0 when the entry is skipped
-// (index out of range or list not strictly ascending). Lengths are clamped to
-// [1, Lmax]. Pure function of global data, so every thread gets the same answer.
-__device__ __forceinline__ int active_len(const Params &p, int i, int U, int &u, int &errbits)
+// Sequence length of unit u, clamped to [1, Lmax] (the prologue reports the
+// clamp; every later lookup must give the same value).
+__device__ __forceinline__ int unit_len(const Params &p, int u)
 {
-    u = __ldg(p.active + 1 + i);
-    const int prev = (i > 0) ? __ldg(p.active + i) : -1;
-    if (u < 0 || u >= U || u <= prev) {
-        errbits |= SR_DEVERR_ACTIVE_LIST;
-        return 0;
+    const int L = __ldg(p.seq_lens + u / p.Hkv);
+    return L < 1 ? 1 : (L > p.Lmax ? p.Lmax : L);
+}
+
+// Smallest set bit >= from in a bitmap of U bits, or U when there is none.
+__device__ __forceinline__ int next_set_bit(const uint32_t *bm, int from, int U)
+{
+    const int nw = (U + 31) >> 5;
+    int w = from >> 5;
+    if (from >= U || w >= nw)
+        return U;
+    uint32_t bits = bm[w] & (0xffffffffu << (from & 31));
+    while (!bits) {
+        if (++w >= nw)
+            return U;
+        bits = bm[w];
     }
-    int L = __ldg(p.seq_lens + u / p.Hkv);
-    if (L < 1 || L > p.Lmax) {
-        errbits |= SR_DEVERR_SEQ_LEN;
-        L = L < 1 ? 1 : p.Lmax;
-    }
-    return L;
+    const int r = (w << 5) + __ffs(bits) - 1;
+    return r < U ? r : U;
 }
 
 // Inclusive block-wide prefix of a 64-bit value; *total receives the block sum.
@@ -188,7 +199,33 @@ __device__ __forceinline__ long long block_scan(long long x, Misc *misc, long lo
     return before + v;
 }
 
-template <int RB, int STAGES>
+// Fused routing, one pass per kThreads (unit, head) pairs: sflag[u] = sink.
+// Every CTA computes the same decisions as the routing kernel (same
+// arithmetic, sr_route_math.cuh); CTA 0 also writes the route mask.
+template <int M>
+__device__ __forceinline__ void route_units(const Params &p, int U, uint8_t *sflag)
+{
+    const int pairs = U * M;
+    for (int base = 0; base < pairs; base += kThreads) {
+        const int pr = base + (int)threadIdx.x;
+        const bool valid = pr < pairs;
+        const int u = pr / M, m = pr - (pr / M) * M;
+        float c = INFINITY;
+        if (valid) {
+            const int b = u / p.Hkv, g = u - b * p.Hkv;
+            c = head_cosine(p.q + ((size_t)b * p.Hq + (size_t)g * M + m) * kHeadDim, p.k0 + (size_t)u * kHeadDim);
+        }
+        c = group_min<M>(c);
+        if (valid && m == 0) {
+            const uint8_t sink = (c >= p.tau) ? 1 : 0;
+            sflag[u] = sink;
+            if (blockIdx.x == 0 && p.mask_out)
+                p.mask_out[u] = sink;
+        }
+    }
+}
+
+template <int RB, int STAGES, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p)
 {
@@ -222,6 +259,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         misc->is_last = 0;
         misc->i0 = INT_MAX;
         misc->s0 = 0;
+        misc->first_bad = INT_MAX;
+        misc->first_u = -1;
     }
     if (warp == kCWarps && lane == 0) {
         prefetch_tensormap(&tmK);
@@ -229,46 +268,107 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     }
     for (int w = tid; w < (U + 31) / 32; w += kThreads)
         bitmap[w] = 0;
+    __syncthreads();
     int32_t *seqtab = reinterpret_cast<int32_t *>(smem);
     int32_t *ltab = seqtab + kSeqTab;
     int16_t *utab = reinterpret_cast<int16_t *>(ltab + SR_MAX_UNITS);
     const bool seq_smem = p.B <= kSeqTab;
-    // seq_lens is a caller input that was complete before the routing kernel
-    // ran, so it is staged before the dependency wait; the active list is the
-    // routing kernel's output and is read only after it.
-    if (seq_smem)
-        for (int b = tid; b < p.B; b += kThreads)
-            seqtab[b] = __ldg(p.seq_lens + b);
-    grid_dependency_wait();
-    grid_launch_dependents();
-    __syncthreads();
-
     int errbits = 0;
-    int n = __ldg(p.active);
-    if (n < 0 || n > U) {
-        errbits |= SR_DEVERR_ACTIVE_LIST;
-        n = n < 0 ? 0 : U;
-    }
+    int n = 0;
     long long local = 0;
-    for (int i = tid; i < U; i += kThreads) {
-        const int u = __ldg(p.active + 1 + i);
-        const int prev = (i > 0) ? __ldg(p.active + i) : -1;
-        if (i >= n)
-            continue;
-        int L = 0;
-        if (u < 0 || u >= U || u <= prev) {
+    if constexpr (!FUSED) {
+        // seq_lens is a caller input that was complete before the routing
+        // kernel ran, so it is staged before the dependency wait; the active
+        // list is the routing kernel's output and is read only after it.
+        if (seq_smem)
+            for (int b = tid; b < p.B; b += kThreads)
+                seqtab[b] = __ldg(p.seq_lens + b);
+        grid_dependency_wait();
+        grid_launch_dependents();
+        __syncthreads();
+
+        n = __ldg(p.active);
+        if (n < 0 || n > U) {
             errbits |= SR_DEVERR_ACTIVE_LIST;
-        } else {
-            L = seq_smem ? seqtab[u / p.Hkv] : __ldg(p.seq_lens + u / p.Hkv);
+            n = n < 0 ? 0 : U;
+        }
+        // Keep the longest well-formed prefix of the list (indices in range and
+        // strictly ascending); a malformed entry ends it and is reported.
+        for (int i = tid; i < U; i += kThreads) {
+            const int u = __ldg(p.active + 1 + i);
+            const int prev = (i > 0) ? __ldg(p.active + i) : -1;
+            if (i >= n)
+                continue;
+            if (u < 0 || u >= U || u <= prev)
+                atomicMin(&misc->first_bad, i);
+            else
+                utab[i] = (int16_t)u;
+        }
+        __syncthreads();
+        if (misc->first_bad < n) {
+            errbits |= SR_DEVERR_ACTIVE_LIST;
+            n = misc->first_bad;
+        }
+        for (int i = tid; i < n; i += kThreads) {
+            const int u = utab[i];
+            int L = seq_smem ? seqtab[u / p.Hkv] : __ldg(p.seq_lens + u / p.Hkv);
             if (L < 1 || L > p.Lmax) {
                 errbits |= SR_DEVERR_SEQ_LEN;
                 L = L < 1 ? 1 : p.Lmax;
             }
             atomicOr(&bitmap[u >> 5], 1u << (u & 31));
+            ltab[i] = L;
+            local += L;
         }
-        ltab[i] = L;
-        utab[i] = (int16_t)(L > 0 ? u : -1);
-        local += L;
+    } else {
+        // Routing inside the kernel: every input may come from the preceding
+        // kernel, so everything is read after the dependency wait.
+        grid_dependency_wait();
+        grid_launch_dependents();
+        uint8_t *sflag = reinterpret_cast<uint8_t *>(utab + SR_MAX_UNITS);
+        if (seq_smem)
+            for (int b = tid; b < p.B; b += kThreads)
+                seqtab[b] = __ldg(p.seq_lens + b);
+        switch (M) {
+        case 1:
+            route_units<1>(p, U, sflag);
+            break;
+        case 2:
+            route_units<2>(p, U, sflag);
+            break;
+        case 4:
+            route_units<4>(p, U, sflag);
+            break;
+        default:
+            route_units<8>(p, U, sflag);
+            break;
+        }
+        __syncthreads();
+        // Ordered compaction of the active units into the same tables the
+        // work-list path builds.
+        for (int c0 = 0; c0 < U; c0 += kThreads) {
+            const int u = c0 + tid;
+            const bool act = (u < U) && !sflag[u];
+            long long tot;
+            const long long incl = block_scan(act ? 1 : 0, misc, &tot);
+            if (act) {
+                const int i = n + (int)incl - 1;
+                int L = seq_smem ? seqtab[u / p.Hkv] : __ldg(p.seq_lens + u / p.Hkv);
+                if (L < 1 || L > p.Lmax) {
+                    errbits |= SR_DEVERR_SEQ_LEN;
+                    L = L < 1 ? 1 : p.Lmax;
+                }
+                atomicOr(&bitmap[u >> 5], 1u << (u & 31));
+                ltab[i] = L;
+                utab[i] = (int16_t)u;
+                local += L;
+                if (blockIdx.x == 0 && p.active_out)
+                    p.active_out[1 + i] = u;
+            }
+            n += (int)tot;
+        }
+        if (blockIdx.x == 0 && tid == 0 && p.active_out)
+            p.active_out[0] = n;
     }
     long long P;
     (void)block_scan(local, misc, &P);
@@ -300,10 +400,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         }
     }
     __syncthreads();
-    if (tid < kUnitCache && misc->i0 < n) {
-        const int i = misc->i0 + tid;
-        misc->cache_u[tid] = (i < n) ? (int)utab[i] : -1;
-        misc->cache_l[tid] = (i < n) ? ltab[i] : 0;
+    if (tid == 0) {
+        // The producer walks the active units in the bitmap from its first
+        // entry on (rank i0 for automatic splits, rank 0 for forced ones).
+        const int i0 = (p.n_splits == 0) ? misc->i0 : 0;
+        misc->i0 = i0;
+        misc->first_u = (i0 < n) ? (int)utab[i0] : -1;
     }
     __syncthreads(); // the stage buffers are free for the copies from here on
 
@@ -371,26 +473,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             return true;
         };
 
+        // Active entry of rank i, for non-decreasing i: ranks follow the set
+        // bits of the bitmap in ascending unit order, starting at first_u.
+        int wi = misc->i0, wu = misc->first_u;
+        auto unit_at = [&](int i) -> int {
+            while (wi < i && wu < U) {
+                wu = next_set_bit(bitmap, wu + 1, U);
+                ++wi;
+            }
+            return wu;
+        };
         if (p.n_splits == 0) {
             if (P > 0 && r0 < P) {
-                const int i0 = misc->i0;
-                int i = i0;
+                int i = misc->i0;
                 long long S = misc->s0;
                 while (ok && i < n && S < r1) {
-                    int u, L;
-                    if (i - i0 < kUnitCache) {
-                        u = misc->cache_u[i - i0];
-                        L = misc->cache_l[i - i0];
-                    } else {
-                        int dummy = 0;
-                        L = active_len(p, i, U, u, dummy);
-                    }
-                    if (L > 0) {
-                        const long long b0 = (r0 > S ? r0 : S) - S;
-                        const long long e0 = (r1 < S + L ? r1 : S + L) - S;
-                        const long long cf = S / chunk, cl = (S + L - 1) / chunk;
-                        ok = emit_split(u, b0, e0, (int)blockIdx.x + i, (int)(cl - cf + 1), (int)cf + i);
-                    }
+                    const int u = unit_at(i);
+                    if (u < 0 || u >= U)
+                        break;
+                    const int L = unit_len(p, u);
+                    const long long b0 = (r0 > S ? r0 : S) - S;
+                    const long long e0 = (r1 < S + L ? r1 : S + L) - S;
+                    const long long cf = S / chunk, cl = (S + L - 1) / chunk;
+                    ok = emit_split(u, b0, e0, (int)blockIdx.x + i, (int)(cl - cf + 1), (int)cf + i);
                     S += L;
                     ++i;
                 }
@@ -399,10 +504,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             const int ns = p.n_splits;
             for (long long j = blockIdx.x; ok && j < (long long)n * ns; j += G) {
                 const int i = (int)(j / ns), s = (int)(j % ns);
-                int u, dummy = 0;
-                const int L = active_len(p, i, U, u, dummy);
-                if (L == 0)
-                    continue;
+                const int u = unit_at(i);
+                if (u < 0 || u >= U)
+                    break;
+                const int L = unit_len(p, u);
                 const long long b0 = (long long)s * L / ns, e0 = (long long)(s + 1) * L / ns;
                 ok = emit_split(u, b0, e0, (int)j, ns, i * ns);
             }
@@ -847,8 +952,12 @@ cudaError_t configure(int dev, DeviceInfo &info)
     cudaError_t e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
-    KernelFn k = decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES>;
+    KernelFn k = decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES, false>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg::ALLOC);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaFuncSetAttribute(decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg::ALLOC);
     if (e != cudaSuccess)
         return e;
     int per_sm = 0;
@@ -915,6 +1024,10 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
     p.M = a.n_q_heads / a.n_kv_heads;
     p.Lmax = a.max_seq_len;
     p.n_splits = a.n_splits;
+    p.k0 = static_cast<const __nv_bfloat16 *>(a.k0);
+    p.tau = a.tau;
+    p.mask_out = a.mask_out;
+    p.active_out = a.active_out;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info->grid);
     cfg.blockDim = dim3(kThreads);
@@ -925,7 +1038,10 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES>, tmK, tmV, p);
+    if (a.fused)
+        e = cudaLaunchKernelEx(&cfg, decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES, true>, tmK, tmV, p);
+    else
+        e = cudaLaunchKernelEx(&cfg, decode_kernel<SR_DECODE_RB, SR_DECODE_STAGES, false>, tmK, tmV, p);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

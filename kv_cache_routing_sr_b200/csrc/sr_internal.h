@@ -58,6 +58,13 @@ struct DecodeArgs {
     void *workspace;
     WorkspaceLayout ws;
     int batch, n_q_heads, n_kv_heads, max_seq_len, n_splits;
+    // Fused routing (sr_route_decode_attention): the kernel routes every unit
+    // itself from q and k0 instead of reading active_list.
+    bool fused = false;
+    const void *k0 = nullptr;
+    float tau = 0.f;
+    uint8_t *mask_out = nullptr;
+    int32_t *active_out = nullptr;
 };
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);

@@ -8,10 +8,10 @@
 // controls -- the threshold is a cosine threshold. The min over heads and ">="
 // are this library's reading of what the pages leave open.
 //
-// Layout: one CTA of 32 warps. Each warp owns whole units (b, g): lane l holds
-// elements 4l..4l+3 of k0_g and of each query head, so a unit's dot products
-// and squared norms are warp shuffle reductions in fp32. All loads of a pass
-// are issued before the first reduction (one memory round trip per pass). The compaction writes
+// Layout: one CTA of 256 threads, one thread per (unit, query head) pair per
+// pass (a pass covers 256 pairs: every workload here routes in one pass). A
+// thread holds both 256-byte rows in registers, so each pass is one memory
+// round trip, and the group minimum is a shuffle over adjacent lanes. The compaction writes
 // active units in ascending order with warp ballots and a block prefix, so no
 // CTA of the decode kernel is ever bound to a sink unit.
 #include <cuda_bf16.h>
@@ -19,42 +19,24 @@
 
 #include "sr_internal.h"
 #include "sr_ptx.cuh"
+#include "sr_route_math.cuh"
 
 namespace sr {
 namespace {
 
-constexpr int kRouteThreads = 1024;
+constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
 
-__device__ __forceinline__ float warp_sum(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-__device__ __forceinline__ void widen4(uint2 raw, float (&v)[4])
-{
-    const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-    const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-    v[0] = fa.x, v[1] = fa.y, v[2] = fb.x, v[3] = fb.y;
-}
-
-__device__ __forceinline__ float dot4(const float (&a)[4], const float (&b)[4])
-{
-    return a[0] * b[0] + a[1] * b[1] + a[2] * b[2] + a[3] * b[3];
-}
-
-// M = query heads per KV head (compile time). Each warp routes UNR units per
-// pass, with every load of those units (k0 and the M query heads) issued before
-// the first reduction, so a pass costs one memory round trip.
+// M = query heads per KV head (compile time). One thread per (unit, head)
+// pair: it loads the head's query row and the unit's k0 row (2 x 256 bytes,
+// all 32 loads in flight at once) and computes the cosine in fp32. The M
+// threads of a unit are adjacent lanes, so the minimum over the group's heads
+// is a shuffle reduction.
 template <int M>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k0, float tau,
              uint8_t *__restrict__ mask, int32_t *__restrict__ active, int B, int Hkv)
 {
-    constexpr int UNR = (8 / M) > 0 ? (8 / M) : 1;
     extern __shared__ uint8_t sink_flag[]; // [B*Hkv]
     __shared__ int32_t warp_cnt[kRouteWarps];
     __shared__ int32_t warp_off[kRouteWarps + 1];
@@ -66,49 +48,23 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
     grid_launch_dependents();
 
     const int U = B * Hkv;
-    const int Hq = Hkv * M;
+    const int pairs = U * M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    for (int base = warp; base < U; base += kRouteWarps * UNR) {
-        uint2 kraw[UNR], qraw[UNR][M];
-#pragma unroll
-        for (int k = 0; k < UNR; ++k) {
-            const int u = base + k * kRouteWarps;
-            kraw[k] = make_uint2(0u, 0u);
-#pragma unroll
-            for (int m = 0; m < M; ++m)
-                qraw[k][m] = make_uint2(0u, 0u);
-            if (u < U) {
-                const int b = u / Hkv, g = u - b * Hkv;
-                kraw[k] = *reinterpret_cast<const uint2 *>(k0 + (size_t)u * kHeadDim + 4 * lane);
-#pragma unroll
-                for (int m = 0; m < M; ++m)
-                    qraw[k][m] = *reinterpret_cast<const uint2 *>(
-                        q + ((size_t)b * Hq + (size_t)g * M + m) * kHeadDim + 4 * lane);
-            }
+    for (int base = 0; base < pairs; base += kRouteThreads) {
+        const int pr = base + (int)threadIdx.x;
+        const bool valid = pr < pairs;
+        const int u = pr / M, m = pr - (pr / M) * M;
+        float c = INFINITY;
+        if (valid) {
+            const int b = u / Hkv, g = u - b * Hkv;
+            c = head_cosine(q + ((size_t)b * Hkv * M + (size_t)g * M + m) * kHeadDim, k0 + (size_t)u * kHeadDim);
         }
-#pragma unroll
-        for (int k = 0; k < UNR; ++k) {
-            const int u = base + k * kRouteWarps;
-            float kv[4];
-            widen4(kraw[k], kv);
-            const float kk = warp_sum(dot4(kv, kv));
-            float s = INFINITY;
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                float qv[4];
-                widen4(qraw[k][m], qv);
-                const float dot = warp_sum(dot4(qv, kv));
-                const float qq = warp_sum(dot4(qv, qv));
-                const float c = (qq == 0.f || kk == 0.f) ? 0.f : dot / (sqrtf(qq) * sqrtf(kk));
-                // A NaN cosine never lowers the minimum (same rule as a "<" scan).
-                s = (c < s) ? c : s;
-            }
-            if (u < U && lane == 0) {
-                const uint8_t sink = (s >= tau) ? 1 : 0;
-                mask[u] = sink;
-                sink_flag[u] = sink;
-            }
+        c = group_min<M>(c); // minimum over the M adjacent lanes of the unit
+        if (valid && m == 0) {
+            const uint8_t sink = (c >= tau) ? 1 : 0;
+            mask[u] = sink;
+            sink_flag[u] = sink;
         }
     }
     __syncthreads();
@@ -124,7 +80,7 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
             warp_cnt[warp] = __popc(ball);
         __syncthreads();
         if (warp == 0) {
-            const int v = warp_cnt[lane];
+            const int v = (lane < kRouteWarps) ? warp_cnt[lane] : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -132,8 +88,9 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
                 if (lane >= o)
                     incl += y;
             }
-            warp_off[lane] = incl - v;
-            if (lane == 31)
+            if (lane < kRouteWarps)
+                warp_off[lane] = incl - v;
+            if (lane == kRouteWarps - 1)
                 warp_off[kRouteWarps] = incl;
         }
         __syncthreads();

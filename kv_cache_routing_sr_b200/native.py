@@ -40,7 +40,7 @@ _lib = None
 
 EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_decode_attention",
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
-           "sr_last_cuda_error", "sr_decode_attention_static_scratch"]
+           "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention"]
 
 
 def load(path: str = LIBRARY):
@@ -74,6 +74,9 @@ def load(path: str = LIBRARY):
     lib.sr_last_cuda_error.restype = ctypes.c_char_p
     lib.sr_decode_attention_static_scratch.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.sr_decode_attention_static_scratch.restype = ctypes.c_int
+    lib.sr_route_decode_attention.argtypes = [dp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, vp, vp,
+                                              u64, vp]
+    lib.sr_route_decode_attention.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -194,6 +197,28 @@ def decode_attention_static_scratch(q, k_cache, v_cache, k0, v0, seq_lens, activ
     return out
 
 
+def route_decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, tau, out=None, route_mask=None,
+                           active_list=None, n_splits: int = 0, workspace: Workspace | None = None, stream=None):
+    """sr_route_decode_attention: routing and decode in one launch. Returns out;
+    route_mask / active_list (optional tensors) receive the route result."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = Workspace(B, Hq, Hkv, Lmax, n_splits, device=q.device)
+    dims = dims_of(B, Hq, Hkv, Lmax, d)
+    mp = _dev(route_mask, "route_mask", torch.uint8) if route_mask is not None else None
+    ap = _dev(active_list, "active_list", torch.int32) if active_list is not None else None
+    st = load().sr_route_decode_attention(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+        _dev(v_cache, "v_cache", torch.bfloat16), _dev(k0, "k0", torch.bfloat16), _dev(v0, "v0", torch.bfloat16),
+        _dev(seq_lens, "seq_lens", torch.int32), float(tau), int(n_splits), mp, ap,
+        _dev(out, "out", torch.bfloat16), ctypes.c_void_p(workspace.ptr), workspace.nbytes, _stream(stream))
+    _check("sr_route_decode_attention", st)
+    return out
+
+
 def grid_size() -> int:
     return int(load().sr_decode_grid_size())
 
@@ -216,3 +241,44 @@ class Decoder:
         decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, self.active_list, self.out, n_splits,
                          self.workspace, stream)
         return self.out
+
+    def step_fused(self, q, k_cache, v_cache, k0, v0, seq_lens, tau, n_splits: int = 0, stream=None):
+        """The same step in one launch (sr_route_decode_attention)."""
+        route_decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, tau, self.out, self.route_mask,
+                               self.active_list, n_splits, self.workspace, stream)
+        return self.out
+
+
+class StepGraph:
+    """One decode step captured in a CUDA graph: sr_route then
+    sr_decode_attention (either may be left out) on fixed tensors, replayed with
+    one graph launch. The programmatic dependency between the two kernels is
+    kept as a graph edge, and the host cost per step is a single launch.
+
+    The tensors are bound at capture: replay reads whatever they hold then."""
+
+    def __init__(self, decoder: "Decoder", q, k_cache, v_cache, k0, v0, seq_lens, tau, n_splits: int = 0,
+                 with_route: bool = True, with_decode: bool = True):
+        self.decoder = decoder
+        self.graph = torch.cuda.CUDAGraph()
+        args = (q, k_cache, v_cache, k0, v0, seq_lens)
+
+        def body():
+            if with_route:
+                route(q, k0, tau, decoder.route_mask, decoder.active_list)
+            if with_decode:
+                decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, decoder.active_list, decoder.out,
+                                 n_splits, decoder.workspace)
+
+        side = torch.cuda.Stream(device=q.device)
+        side.wait_stream(torch.cuda.current_stream(q.device))
+        with torch.cuda.stream(side):  # warm-up outside the capture (module load, attributes)
+            decoder.step(*args, tau, n_splits)
+        torch.cuda.current_stream(q.device).wait_stream(side)
+        with torch.cuda.graph(self.graph):
+            body()
+        self._args = args  # keep the bound tensors alive as long as the graph
+
+    def replay(self):
+        self.graph.replay()
+        return self.decoder.out

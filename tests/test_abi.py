@@ -109,3 +109,19 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(native, "_lib", None)
     with pytest.raises(RuntimeError, match="not found"):
         native.load(str(tmp_path / "nope.so"))
+
+
+def test_fused_entry_validation(lib):
+    d = dims()
+    c = lambda **kw: lib.sr_route_decode_attention(  # noqa: E731
+        ctypes.byref(d), FAKE, FAKE, FAKE, kw.get("k0", FAKE), FAKE, FAKE, ctypes.c_float(kw.get("tau", 0.6)),
+        kw.get("ns", 0), None, kw.get("act", None), FAKE, kw.get("ws", FAKE), kw.get("wsb", 1 << 30), None)
+    assert c(k0=None) == native.SR_ERR_INVALID_ARG  # the fused call routes, so k0 is required
+    assert c(tau=float("nan")) == native.SR_ERR_INVALID_ARG
+    assert c(act=FAKE + 2) == native.SR_ERR_INVALID_ARG
+    assert c(ns=-3) == native.SR_ERR_INVALID_ARG
+    assert c(ws=None) == native.SR_ERR_WORKSPACE
+    assert c(wsb=16) == native.SR_ERR_WORKSPACE
+    bad = dims(d=96)
+    assert lib.sr_route_decode_attention(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.6),
+                                         0, None, None, FAKE, FAKE, 1 << 30, None) == native.SR_ERR_UNSUPPORTED

@@ -205,3 +205,66 @@ def test_bad_active_list_is_reported_not_fatal():
     torch.cuda.synchronize()
     assert dec.workspace.device_error() & native.SR_DEVERR_ACTIVE_LIST
     assert torch.isfinite(dec.out.float()).all()
+
+
+def test_step_graph_replay_matches_eager_and_tracks_inputs():
+    """A captured step (route + decode in one CUDA graph) gives the eager result,
+    and replays read the bound tensors' current contents."""
+    x = inputs.make("llama70b_ragged", seed=23, device=DEV, max_ctx=2000)
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    eager = dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau).clone()
+    mask_e = dec.route_mask.clone()
+    g = native.StepGraph(dec, x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+    for _ in range(2):
+        out = g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager) and torch.equal(dec.route_mask, mask_e)
+    # change the inputs in place: make every group of sequence 0 a sink
+    x.q[0] = x.k0[0].repeat_interleave(8, dim=0)
+    out = g.replay().cpu()
+    torch.cuda.synchronize()
+    mask = dec.route_mask.cpu()
+    assert bool(mask[:8].all())
+    H.check_against_oracle(x, out, mask)
+
+
+# ---- fused routing + decode (one launch) -------------------------------------------------
+
+FUSED_CASES = [
+    ("tiny_4k", {}),
+    ("llama8b_128k", dict(max_ctx=5000)),
+    ("llama70b_ragged", dict(max_ctx=3000, poison_padding=True)),
+    ("llava7b_mha", dict(max_ctx=1500)),
+    ("llama8b_512k", dict(max_ctx=2048, sink_fraction=1.0)),
+    ("llama8b_512k", dict(max_ctx=2048, sink_fraction=0.0)),
+]
+
+
+@pytest.mark.parametrize("name,kw", FUSED_CASES, ids=[f"{c[0]}-{i}" for i, c in enumerate(FUSED_CASES)])
+def test_fused_step_equals_two_calls(name, kw):
+    x = inputs.make(name, seed=31, device=DEV, **kw)
+    two = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    one = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    for ns in (0, 3):
+        ref = two.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau, n_splits=0 if ns == 0 else ns)
+        got = one.step_fused(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau,
+                             n_splits=0 if ns == 0 else ns)
+        torch.cuda.synchronize()
+        assert torch.equal(one.route_mask, two.route_mask)
+        n = int(two.active_list[0])
+        assert torch.equal(one.active_list[:1 + n], two.active_list[:1 + n])
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), "fused output differs from two calls"
+    assert one.workspace.device_error() == 0
+    H.check_against_oracle(x, got.cpu(), one.route_mask.cpu())
+
+
+def test_fused_full_size_and_optional_outputs():
+    x = inputs.make("llama8b_128k", seed=0, device=DEV)
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    out = native.route_decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau,
+                                        workspace=dec.workspace)  # no route outputs requested
+    torch.cuda.synchronize()
+    mask_r, _, _ = oracle.route(x.q.cpu(), x.k0.cpu(), H.tau32(x.tau))
+    H.check_against_oracle(x, out.cpu(), mask_r, units=[0, 3, 4, 7])
+    g = native.StepGraph(dec, x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+    assert torch.equal(g.replay(), out)
