@@ -213,7 +213,8 @@ __device__ __forceinline__ void route_units(const Params &p, int U, uint8_t *sfl
         float c = INFINITY;
         if (valid) {
             const int b = u / p.Hkv, g = u - b * p.Hkv;
-            c = head_cosine(p.q + ((size_t)b * p.Hq + (size_t)g * M + m) * kHeadDim, p.k0 + (size_t)u * kHeadDim);
+            c = head_cosine(p.q + ((size_t)b * p.Hq + (size_t)g * M + m) * kHeadDim, p.k0 + (size_t)u * kHeadDim,
+                            pr & 15);
         }
         c = group_min<M>(c);
         if (valid && m == 0) {
@@ -269,10 +270,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     for (int w = tid; w < (U + 31) / 32; w += kThreads)
         bitmap[w] = 0;
     __syncthreads();
-    int32_t *seqtab = reinterpret_cast<int32_t *>(smem);
-    int32_t *ltab = seqtab + kSeqTab;
-    int16_t *utab = reinterpret_cast<int16_t *>(ltab + SR_MAX_UNITS);
+    // Prologue tables in the stage buffers (free until the first copy),
+    // sized by the actual batch and unit count.
     const bool seq_smem = p.B <= kSeqTab;
+    const int seq_bytes = seq_smem ? ((4 * p.B + 127) & ~127) : 0;
+    int32_t *seqtab = reinterpret_cast<int32_t *>(smem);
+    int32_t *ltab = reinterpret_cast<int32_t *>(smem + seq_bytes);
+    int16_t *utab = reinterpret_cast<int16_t *>(smem + seq_bytes + ((4 * U + 127) & ~127));
+    uint8_t *sflag = smem + seq_bytes + ((4 * U + 127) & ~127) + ((2 * U + 127) & ~127);
     int errbits = 0;
     int n = 0;
     long long local = 0;
@@ -325,10 +330,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         // kernel, so everything is read after the dependency wait.
         grid_dependency_wait();
         grid_launch_dependents();
-        uint8_t *sflag = reinterpret_cast<uint8_t *>(utab + SR_MAX_UNITS);
         if (seq_smem)
             for (int b = tid; b < p.B; b += kThreads)
                 seqtab[b] = __ldg(p.seq_lens + b);
+        // One thread per (unit, head) pair reads both rows straight from
+        // global memory. (Staging them with bulk copies in every CTA was
+        // measured slower: 148 CTAs copying the same few KB serialise.)
         switch (M) {
         case 1:
             route_units<1>(p, U, sflag);
@@ -399,6 +406,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             }
         }
     }
+    // Generic stores into the stage buffers (tables) must be ordered before
+    // the TMA writes that will reuse those bytes.
+    fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
         // The producer walks the active units in the bitmap from its first

@@ -8,15 +8,17 @@
 // controls -- the threshold is a cosine threshold. The min over heads and ">="
 // are this library's reading of what the pages leave open.
 //
-// Layout: one CTA of 256 threads, one thread per (unit, query head) pair per
-// pass (a pass covers 256 pairs: every workload here routes in one pass). A
-// thread holds both 256-byte rows in registers, so each pass is one memory
-// round trip, and the group minimum is a shuffle over adjacent lanes. The compaction writes
+// Layout: one CTA of 256 threads. The q and k0 rows of a chunk of units (all
+// units, for every workload here) are staged in shared memory by two bulk
+// copies, then one thread per (unit, query head) pair computes the cosine and
+// the group minimum is a shuffle over adjacent lanes. The compaction writes
 // active units in ascending order with warp ballots and a block prefix, so no
 // CTA of the decode kernel is ever bound to a sink unit.
+#include <atomic>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "sinkrouter.h"
 #include "sr_internal.h"
 #include "sr_ptx.cuh"
 #include "sr_route_math.cuh"
@@ -27,47 +29,77 @@ namespace {
 constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
 
-// M = query heads per KV head (compile time). One thread per (unit, head)
-// pair: it loads the head's query row and the unit's k0 row (2 x 256 bytes,
-// all 32 loads in flight at once) and computes the cosine in fp32. The M
-// threads of a unit are adjacent lanes, so the minimum over the group's heads
-// is a shuffle reduction.
+constexpr int kRowBudget = 160 * 1024; // shared bytes for staged q / k0 rows
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Units per staged chunk for group size M.
+template <int M> constexpr int chunk_units() { return kRowBudget / ((M + 1) * 256); }
+
+// M = query heads per KV head (compile time). The q rows of a chunk of units
+// and their k0 rows are contiguous in global memory, so one thread stages them
+// with two bulk copies (one memory round trip, whatever the chunk size); then
+// one thread per (unit, head) pair computes the cosine from shared memory and
+// the M lanes of a unit take the minimum with shuffles.
 template <int M>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k0, float tau,
-             uint8_t *__restrict__ mask, int32_t *__restrict__ active, int B, int Hkv)
+             uint8_t *__restrict__ mask, int32_t *__restrict__ active, int B, int Hkv, int cu)
 {
-    extern __shared__ uint8_t sink_flag[]; // [B*Hkv]
+    extern __shared__ __align__(128) uint8_t dsm[]; // [cu*(M+1)*256 staged rows][B*Hkv sink flags]
+    __shared__ __align__(8) uint64_t bar;
     __shared__ int32_t warp_cnt[kRouteWarps];
     __shared__ int32_t warp_off[kRouteWarps + 1];
 
+    const int U = B * Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint4 *rows = reinterpret_cast<uint4 *>(dsm);
+    uint8_t *sink_flag = dsm + (size_t)cu * (M + 1) * 256;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_mbar_init();
+    }
     // Inputs may come from the previous kernel in the stream, and the previous
     // decode step may still read route_mask / active_list: wait for it, then
     // let the decode kernel that follows launch and run its prologue.
     grid_dependency_wait();
     grid_launch_dependents();
-
-    const int U = B * Hkv;
-    const int pairs = U * M;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    for (int base = 0; base < pairs; base += kRouteThreads) {
-        const int pr = base + (int)threadIdx.x;
-        const bool valid = pr < pairs;
-        const int u = pr / M, m = pr - (pr / M) * M;
-        float c = INFINITY;
-        if (valid) {
-            const int b = u / Hkv, g = u - b * Hkv;
-            c = head_cosine(q + ((size_t)b * Hkv * M + (size_t)g * M + m) * kHeadDim, k0 + (size_t)u * kHeadDim);
-        }
-        c = group_min<M>(c); // minimum over the M adjacent lanes of the unit
-        if (valid && m == 0) {
-            const uint8_t sink = (c >= tau) ? 1 : 0;
-            mask[u] = sink;
-            sink_flag[u] = sink;
-        }
-    }
     __syncthreads();
+
+    uint32_t ph = 0;
+    bool timed_out = false;
+    for (int u0 = 0; u0 < U; u0 += cu) {
+        const int nu = (U - u0) < cu ? (U - u0) : cu;
+        if (threadIdx.x == 0) {
+            const uint32_t qbytes = (uint32_t)nu * M * 256, kbytes = (uint32_t)nu * 256;
+            mbar_arrive_expect_tx(b, qbytes + kbytes);
+            bulk_load(smem_u32(rows), q + (size_t)u0 * M * kHeadDim, qbytes, b);
+            bulk_load(smem_u32(rows) + qbytes, k0 + (size_t)u0 * kHeadDim, kbytes, b);
+        }
+        if (!mbar_try_wait(b, ph)) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(b, ph)) {
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                    timed_out = true;
+                    break;
+                }
+            }
+        }
+        ph ^= 1;
+        if (__syncthreads_or(timed_out)) {
+            timed_out = true;
+            break;
+        }
+        route_staged<M, kRouteThreads>(rows, u0, nu, tau, sink_flag, mask);
+        __syncthreads(); // the rows are overwritten by the next chunk
+    }
+    if (timed_out) {
+        // A copy never completed (never expected): publish an invalid count,
+        // which the decode kernel reports as SR_DEVERR_ACTIVE_LIST.
+        if (threadIdx.x == 0)
+            active[0] = -1;
+        return;
+    }
 
     // Ordered compaction of the active units.
     int32_t total = 0;
@@ -106,10 +138,25 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
 template <int M>
 cudaError_t launch_route_m(const RouteArgs &a, cudaStream_t stream)
 {
+    const int U = a.batch * a.n_kv_heads;
+    const int cu = U < chunk_units<M>() ? U : chunk_units<M>();
+    const size_t smem = (size_t)cu * (M + 1) * 256 + (size_t)U;
+    static std::atomic<bool> configured[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < 64 && !configured[dev].load()) {
+        e = cudaFuncSetAttribute(route_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)((size_t)chunk_units<M>() * (M + 1) * 256 + SR_MAX_UNITS));
+        if (e != cudaSuccess)
+            return e;
+        configured[dev].store(true);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kRouteThreads);
-    cfg.dynamicSmemBytes = (size_t)a.batch * a.n_kv_heads;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -118,7 +165,7 @@ cudaError_t launch_route_m(const RouteArgs &a, cudaStream_t stream)
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, route_kernel<M>, static_cast<const __nv_bfloat16 *>(a.q),
                               static_cast<const __nv_bfloat16 *>(a.k0), a.tau, a.mask, a.active, a.batch,
-                              a.n_kv_heads);
+                              a.n_kv_heads, cu);
 }
 
 } // namespace
