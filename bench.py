@@ -59,6 +59,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the 512K sink-fraction sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--multilayer", action="store_true",
+                    help="instead of the contract line: per-token attention latency of a 32-layer stack, "
+                         "CUDA-graph captured, at 128K/256K/512K context, routed vs routing disabled")
+    ap.add_argument("--layers", type=int, default=32)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -266,9 +270,9 @@ def time_kernels(native, dec, x, tau, steps, flush):
     return [e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev]
 
 
-def measure_workload(native, inputs, x, steps, warmup, flush, barrier, two_call=True):
-    """Timings of one workload on this GPU: the fused step (routed and with
-    routing disabled) and, if asked, the two-call step and its kernels."""
+def measure_workload(native, inputs, x, steps, warmup, flush, barrier, fused=True):
+    """Timings of one workload on this GPU: the two-call step (routed and with
+    routing disabled) and its kernels, and, if asked, the fused step."""
     import torch
     dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
     for _ in range(warmup):
@@ -282,12 +286,12 @@ def measure_workload(native, inputs, x, steps, warmup, flush, barrier, two_call=
     sl = x.seq_lens.cpu().tolist()
     r = dict(dec=dec, active=act, need=inputs.needed_bytes(sl, act, x.n_kv_heads, x.n_q_heads, x.batch),
              need_all=inputs.needed_bytes(sl, range(x.batch * x.n_kv_heads), x.n_kv_heads, x.n_q_heads, x.batch))
-    r["fused"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, True)
-    r["fused_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, True)
-    if two_call:
-        r["two"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, False)
-        r["route"], r["decode"] = time_kernels(native, dec, x, x.tau, steps, flush)
-        r["two_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, False)
+    r["two"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, False)
+    r["route"], r["decode"] = time_kernels(native, dec, x, x.tau, steps, flush)
+    r["two_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, False)
+    if fused:
+        r["fused"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, True)
+        r["fused_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, True)
     err = dec.workspace.device_error()
     if err:
         raise RuntimeError(f"device error word {err} after the timed steps")
@@ -440,12 +444,14 @@ def run_ours(args):
         for frac in (0.0, 0.25, 0.5, 0.75, 1.0):
             x5 = inputs.make("llama8b_512k", seed=args.seed, device=dev, sink_fraction=frac)
             s5 = measure_workload(native, inputs, x5, max(20, min(K, 50)), args.warmup, flush, barrier,
-                                  two_call=False)
-            u5 = statistics.mean(s5["fused"]) * 1e3
-            ud5 = statistics.mean(s5["fused_disabled"]) * 1e3
+                                  fused=False)
+            u5 = statistics.mean(s5["two"]) * 1e3
+            ud5 = statistics.mean(s5["two_disabled"]) * 1e3
+            d5 = statistics.mean(s5["decode"]) * 1e3
             sweep.append({"sink_fraction": frac, "us_per_layer_step": round(u5, 2),
                           "effective_gbs": round(s5["need"] / (u5 * 1e-6) / 1e9, 1),
                           "frac_of_peak": round(s5["need"] / (u5 * 1e-6) / 1e9 / peak, 4),
+                          "decode_kernel_gbs": round(s5["need"] / (d5 * 1e-6) / 1e9, 1),
                           "routing_disabled_us": round(ud5, 2), "speedup_routed": round(ud5 / u5, 3)})
             del x5, s5
             torch.cuda.empty_cache()
@@ -526,8 +532,58 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_multilayer(args):
+    """Per-token attention latency of an n-layer Llama-3.1-8B-shaped stack (each
+    layer its own 4-of-8-sinks inputs and cache), one CUDA graph per token."""
+    import torch
+
+    from kv_cache_routing_sr_b200 import multilayer
+    peak, peak_kind = hbm_peak()
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    rows = []
+    for ctx in (131072, 262144, 524288):
+        stack = multilayer.LayerStack("llama8b_512k", args.layers, seed=args.seed, max_ctx=ctx,
+                                      sink_fraction=0.5)
+        res = {"context": ctx, "layers": args.layers}
+        for key, gate in (("routed_all_layers", multilayer.LayerGate(0, args.layers - 1)),
+                          ("routed_layers_8_to_end", multilayer.LayerGate(8, args.layers - 1)),
+                          ("routing_disabled", multilayer.LayerGate(1, 0))):
+            g = stack.capture(gate)
+            for _ in range(args.warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            need = stack.needed_bytes()
+            st = torch.cuda.current_stream()
+            times = []
+            for _ in range(max(5, min(args.steps, 20))):
+                flush.sum()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                g.replay()
+                e1.record(st)
+                e1.synchronize()
+                times.append(e0.elapsed_time(e1) * 1e3)
+            us = statistics.median(times)
+            res[key] = {"us_per_token": round(us, 1), "effective_gbs": round(need / (us * 1e-6) / 1e9, 1),
+                        "frac_of_hbm_peak": round(need / (us * 1e-6) / 1e9 / peak, 4),
+                        "active_fraction": round(stack.active_fraction(), 4)}
+            del g
+        res["speedup_all_layers"] = round(res["routing_disabled"]["us_per_token"] /
+                                          res["routed_all_layers"]["us_per_token"], 3)
+        rows.append(res)
+        del stack
+        torch.cuda.empty_cache()
+    print(json.dumps({"measurement": "per-token attention latency, layer stack in one CUDA graph",
+                      "workload": "Llama-3.1-8B-shaped layers (32 q / 8 kv heads, head_dim 128, bf16), batch 1, "
+                                  "4 of 8 groups planted sinks per layer, tau 0.6",
+                      "peak_gbs": peak, "peak_source": f"{peak_kind} HBM copy", "rows": rows}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.multilayer:
+        run_multilayer(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -7,7 +7,7 @@ call into ``native`` does, and raises if it is missing or cannot run.
 """
 from importlib import import_module
 
-__all__ = ["native", "inputs"]
+__all__ = ["native", "inputs", "multilayer"]
 
 
 def __getattr__(name):

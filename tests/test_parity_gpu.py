@@ -268,3 +268,24 @@ def test_fused_full_size_and_optional_outputs():
     H.check_against_oracle(x, out.cpu(), mask_r, units=[0, 3, 4, 7])
     g = native.StepGraph(dec, x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
     assert torch.equal(g.replay(), out)
+
+
+def test_layer_stack_graph_and_gating():
+    """A 4-layer stack in one CUDA graph: replay equals the eager steps, layers
+    outside the gate route nothing, and each layer matches the oracle."""
+    from kv_cache_routing_sr_b200 import multilayer
+    stack = multilayer.LayerStack("llama8b_128k", 4, seed=5, max_ctx=1500)
+    gate = multilayer.LayerGate(1, 2)
+    eager = [o.clone() for o in stack.step_eager(gate)]
+    masks = [dec.route_mask.clone() for _, dec in stack.layers]
+    g = stack.capture(gate)
+    g.replay()
+    torch.cuda.synchronize()
+    for i, ((x, dec), ref) in enumerate(zip(stack.layers, eager)):
+        assert torch.equal(dec.out, ref)
+        assert torch.equal(dec.route_mask, masks[i])
+        if i in (0, 3):
+            assert int(dec.route_mask.sum()) == 0  # gated out: standard attention
+        else:
+            assert int(dec.route_mask.sum()) == 4
+        H.check_against_oracle(x, dec.out.cpu(), dec.route_mask.cpu())
