@@ -63,6 +63,9 @@ def parse_args(argv=None):
                     help="instead of the contract line: per-token attention latency of a 32-layer stack, "
                          "CUDA-graph captured, at 128K/256K/512K context, routed vs routing disabled")
     ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--proxy-quality", action="store_true",
+                    help="instead of the contract line: precision / recall / F1 of the cosine routing proxy "
+                         "against the full-attention position-0 weight, on graded synthetic inputs")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -579,8 +582,27 @@ def run_multilayer(args):
                       "peak_gbs": peak, "peak_source": f"{peak_kind} HBM copy", "rows": rows}), flush=True)
 
 
+def run_proxy_quality(args):
+    """Sweep the routing threshold on graded synthetic decode steps (2048 units,
+    context 16K) and report precision / recall / F1 against the full-attention
+    sink event at three cutoffs."""
+    from kv_cache_routing_sr_b200 import inputs, proxy_quality
+    taus = [round(0.05 * i, 2) for i in range(0, 20)]
+    x = inputs.make_graded(seed=args.seed, batch=256, n_kv_heads=8, group=4, ctx=16384, device="cuda")
+    out = {"measurement": "routing proxy vs full-attention sink event (graded synthetic steps)",
+           "workload": "batch 256 x 8 KV groups x 4 query heads, context 16384, sink strength t ~ U(0,1)",
+           "results": []}
+    for cutoff in (0.5, 0.8, 0.95):
+        res = proxy_quality.evaluate(x, taus, cutoff=cutoff)
+        out["results"].append(res)
+    print(json.dumps(out), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.proxy_quality:
+        run_proxy_quality(args)
+        return
     if args.multilayer:
         run_multilayer(args)
         return

@@ -147,6 +147,26 @@ sr_status sr_decode_attention(const sr_dims *dims, const void *q, const void *k_
                               size_t workspace_bytes, void *stream);
 
 /*
+ * sr_decode_attention_lse -- sr_decode_attention that also returns, for every
+ * query head of an active unit, the natural-log log-sum-exp of its scaled
+ * logits over positions 0 .. L_b-1:
+ *     lse[b, h] = log sum_j exp(<q_h, K[b, g, j]> / sqrt(d))
+ * so that any attention weight can be recovered, e.g. the weight of position 0
+ * p0 = exp(<q_h, K[b, g, 0]> / sqrt(d) - lse[b, h]). The pith.science review of
+ * arXiv 2604.16883 (Figure 10 caption) defines the routing proxy's reference
+ * event from these full-attention position-0 weights. Sink heads get NaN (no
+ * attention is computed for them).
+ *
+ *   lse   out fp32 [B, Hq], device, 4-byte aligned
+ * Other arguments, results and errors: as sr_decode_attention.
+ */
+sr_status sr_decode_attention_lse(const sr_dims *dims, const void *q, const void *k_cache,
+                                  const void *v_cache, const void *k0, const void *v0,
+                                  const int32_t *seq_lens, const int32_t *active_list,
+                                  int32_t n_splits, void *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
+/*
  * sr_route_decode_attention -- sr_route followed by sr_decode_attention in ONE
  * kernel launch: every CTA of the decode kernel routes all units itself (the
  * same fp32 arithmetic as sr_route, so the decisions are identical) and builds

@@ -132,6 +132,37 @@ sr_status sr_decode_attention(const sr_dims *dims, const void *q, const void *k_
     return e == cudaSuccess ? SR_OK : cuda_fail(e);
 }
 
+sr_status sr_decode_attention_lse(const sr_dims *dims, const void *q, const void *k_cache, const void *v_cache,
+                                  const void *k0, const void *v0, const int32_t *seq_lens, const int32_t *active_list,
+                                  int32_t n_splits, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                  void *stream)
+{
+    (void)k0;
+    const sr_status st = check_dims(dims);
+    if (st != SR_OK)
+        return st;
+    if (!q || !k_cache || !v_cache || !v0 || !seq_lens || !active_list || !out || !lse)
+        return SR_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(v0, 16) ||
+        !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(active_list, 4) || !aligned(lse, 4))
+        return SR_ERR_INVALID_ARG;
+    if (n_splits < 0 || n_splits > SR_MAX_SPLITS)
+        return SR_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256))
+        return SR_ERR_WORKSPACE;
+    const int U = dims->batch * dims->n_kv_heads;
+    const int M = dims->n_q_heads / dims->n_kv_heads;
+    const sr::WorkspaceLayout ws = sr::workspace_layout(U, M, sr::slots_needed(U, n_splits));
+    if (workspace_bytes < ws.total)
+        return SR_ERR_WORKSPACE;
+    sr::DecodeArgs a{q,   k_cache,      v_cache,         v0,         seq_lens,         active_list,
+                     out, workspace,    ws,              dims->batch, dims->n_q_heads, dims->n_kv_heads,
+                     dims->max_seq_len, n_splits};
+    a.lse = lse;
+    const cudaError_t e = sr::launch_decode(a, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
 sr_status sr_route_decode_attention(const sr_dims *dims, const void *q, const void *k_cache, const void *v_cache,
                                     const void *k0, const void *v0, const int32_t *seq_lens, float tau,
                                     int32_t n_splits, uint8_t *route_mask, int32_t *active_list, void *out,

@@ -64,6 +64,7 @@ constexpr long long kMinChunk = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull; // 2 s: far above any legitimate wait
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeThreads = 32 * kCWarps;
 constexpr int kMergeBatch = 16; // partials in flight per thread in the final merge
 
@@ -107,6 +108,7 @@ struct Params {
     float tau;
     uint8_t *mask_out;   // may be null
     int32_t *active_out; // may be null
+    float *lse;          // [B, Hq] natural-log log-sum-exp of the logits; may be null
 };
 
 template <int RB, int STAGES> struct Cfg {
@@ -557,6 +559,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + (e >> 4)) * kHeadDim);
                 dst[e & 15] = v;
             }
+            if (p.lse && lane < M) // no attention was computed for a sink head
+                p.lse[(size_t)b * p.Hq + (size_t)gg * M + lane] = __int_as_float(0x7fc00000);
         }
     }
 
@@ -852,6 +856,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         }
                     }
                     if (sgrp == 1) {
+                        if (p.lse && d4 == 0)
+                            p.lse[(size_t)b * p.Hq + (size_t)gg * M + head] = (m + log2f(l)) * kLn2;
                         const float inv = 1.f / l;
                         uint2 packed;
                         packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
@@ -883,6 +889,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                             l += ml.y * c;
                             acc.x += y.x * c, acc.y += y.y * c, acc.z += y.z * c, acc.w += y.w * c;
                         }
+                        if (p.lse && d4 == 0)
+                            p.lse[(size_t)b * p.Hq + (size_t)gg * M + head] = (m + log2f(l)) * kLn2;
                         const float inv = 1.f / l;
                         uint2 packed;
                         packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
@@ -1038,6 +1046,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
     p.tau = a.tau;
     p.mask_out = a.mask_out;
     p.active_out = a.active_out;
+    p.lse = a.lse;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info->grid);
     cfg.blockDim = dim3(kThreads);

@@ -65,6 +65,8 @@ struct DecodeArgs {
     float tau = 0.f;
     uint8_t *mask_out = nullptr;
     int32_t *active_out = nullptr;
+    // Optional per-head log-sum-exp output (sr_decode_attention_lse).
+    float *lse = nullptr;
 };
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);

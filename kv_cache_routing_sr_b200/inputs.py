@@ -33,7 +33,7 @@ IMAGE_TOKENS = 576
 IMAGE_SCALE = 1.5
 
 # Seed offsets per tensor role, so each role has its own stream.
-_ROLE = {"k": 1, "v": 2, "k0dir": 3, "qnoise": 4, "qactive": 5, "lens": 6, "sinks": 7}
+_ROLE = {"k": 1, "v": 2, "k0dir": 3, "qnoise": 4, "qactive": 5, "lens": 6, "sinks": 7, "strength": 8}
 
 
 @dataclass(frozen=True)
@@ -216,6 +216,33 @@ def make(name: str, seed: int = 0, device="cpu", *, max_ctx: int | None = None,
     return DecodeInputs(w, seed, q, k_cache, v_cache, k0, v0, seq_lens.to(device), planted, t)
 
 
+def make_graded(seed: int = 0, device="cpu", *, batch: int = 16, n_kv_heads: int = 8, group: int = 4,
+                ctx: int = 4096, tau: float = 0.6) -> DecodeInputs:
+    """Decode steps with a continuum of sink strength, for studying the routing
+    proxy against full attention. Every unit (b, g) draws a strength t ~ U(0, 1):
+    its position-0 key is k0 = (4 + 36 t) u for a random unit direction u, and
+    each query head is q_h = 40 t u + r_h with r_h ~ N(0, I). Weak units look like
+    ordinary heads (small cosine to k0, small weight on position 0); strong ones
+    like planted sinks. ``extra["strength"]`` holds t [B, Hkv]."""
+    device = torch.device(device)
+    B, Hkv, M, d = batch, n_kv_heads, group, HEAD_DIM
+    Hq = Hkv * M
+    k_cache = torch.empty((B, Hkv, ctx, d), dtype=torch.bfloat16, device=device)
+    v_cache = torch.empty((B, Hkv, ctx, d), dtype=torch.bfloat16, device=device)
+    _fill_normal_bf16(k_cache, _gen(seed, "k", device))
+    _fill_normal_bf16(v_cache, _gen(seed, "v", device))
+    t = torch.rand((B, Hkv), generator=_gen(seed, "strength", device), device=device)
+    u = torch.randn((B, Hkv, d), generator=_gen(seed, "k0dir", device), device=device)
+    u = u / u.norm(dim=-1, keepdim=True)
+    k_cache[:, :, 0] = ((4.0 + 36.0 * t).unsqueeze(-1) * u).to(torch.bfloat16)
+    r = torch.randn((B, Hq, d), generator=_gen(seed, "qnoise", device), device=device)
+    q = ((40.0 * t).repeat_interleave(M, dim=1).unsqueeze(-1) * u.repeat_interleave(M, dim=1) + r)
+    seq_lens = torch.full((B,), ctx, dtype=torch.int32, device=device)
+    w = Workload("graded", B, ctx, Hkv, M, tau=tau, description="graded sink strength t ~ U(0,1) per unit")
+    return DecodeInputs(w, seed, q.to(torch.bfloat16), k_cache, v_cache, k_cache[:, :, 0].clone(),
+                        v_cache[:, :, 0].clone(), seq_lens, t > 0.5, tau, extra={"strength": t})
+
+
 def needed_bytes(seq_lens, active_units, n_kv_heads: int, n_q_heads: int, batch: int,
                  head_dim: int = HEAD_DIM) -> int:
     """Bytes a routed decode step must move: the active groups' K and V rows,
@@ -236,5 +263,5 @@ def describe(name: str) -> str:
     return WORKLOADS[name].description
 
 
-__all__ = ["WORKLOADS", "Workload", "DecodeInputs", "make", "needed_bytes", "describe",
+__all__ = ["WORKLOADS", "Workload", "DecodeInputs", "make", "make_graded", "needed_bytes", "describe",
            "expected_active_fraction", "HEAD_DIM"]

@@ -40,7 +40,8 @@ _lib = None
 
 EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_decode_attention",
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
-           "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention"]
+           "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention",
+           "sr_decode_attention_lse"]
 
 
 def load(path: str = LIBRARY):
@@ -77,6 +78,8 @@ def load(path: str = LIBRARY):
     lib.sr_route_decode_attention.argtypes = [dp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, vp, vp,
                                               u64, vp]
     lib.sr_route_decode_attention.restype = ctypes.c_int
+    lib.sr_decode_attention_lse.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, u64, vp]
+    lib.sr_decode_attention_lse.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -155,8 +158,10 @@ def route(q: torch.Tensor, k0: torch.Tensor, tau: float, route_mask=None, active
 
 
 def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=None, n_splits: int = 0,
-                     workspace: Workspace | None = None, stream=None):
-    """sr_decode_attention: returns out bf16 [B, Hq, 128]."""
+                     workspace: Workspace | None = None, stream=None, lse=None):
+    """sr_decode_attention: returns out bf16 [B, Hq, 128]. With ``lse`` (an fp32
+    CUDA tensor [B, Hq]) it calls sr_decode_attention_lse, which also writes the
+    per-head log-sum-exp of the logits (NaN for sink heads)."""
     B, Hq, d = q.shape
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
     if out is None:
@@ -165,13 +170,16 @@ def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=Non
         workspace = Workspace(B, Hq, Hkv, Lmax, n_splits, device=q.device)
     dims = dims_of(B, Hq, Hkv, Lmax, d)
     k0p = _dev(k0, "k0", torch.bfloat16) if k0 is not None else None
-    st = load().sr_decode_attention(
-        ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
-        _dev(v_cache, "v_cache", torch.bfloat16), k0p, _dev(v0, "v0", torch.bfloat16),
-        _dev(seq_lens, "seq_lens", torch.int32), _dev(active_list, "active_list", torch.int32),
-        int(n_splits), _dev(out, "out", torch.bfloat16), ctypes.c_void_p(workspace.ptr), workspace.nbytes,
-        _stream(stream))
-    _check("sr_decode_attention", st)
+    common = (ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+              _dev(v_cache, "v_cache", torch.bfloat16), k0p, _dev(v0, "v0", torch.bfloat16),
+              _dev(seq_lens, "seq_lens", torch.int32), _dev(active_list, "active_list", torch.int32),
+              int(n_splits), _dev(out, "out", torch.bfloat16))
+    tail = (ctypes.c_void_p(workspace.ptr), workspace.nbytes, _stream(stream))
+    if lse is None:
+        _check("sr_decode_attention", load().sr_decode_attention(*common, *tail))
+    else:
+        _check("sr_decode_attention_lse",
+               load().sr_decode_attention_lse(*common, _dev(lse, "lse", torch.float32), *tail))
     return out
 
 

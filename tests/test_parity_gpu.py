@@ -4,8 +4,10 @@ v0 bit for bit; active outputs within the tolerances of tests/gpu_helpers.py."""
 import pytest
 import torch
 
+import math
+
 import oracle
-from kv_cache_routing_sr_b200 import inputs, native
+from kv_cache_routing_sr_b200 import inputs, native, proxy_quality
 from tests import gpu_helpers as H
 from tests.conftest import cuda_available
 
@@ -289,3 +291,113 @@ def test_layer_stack_graph_and_gating():
         else:
             assert int(dec.route_mask.sum()) == 4
         H.check_against_oracle(x, dec.out.cpu(), dec.route_mask.cpu())
+
+
+# ---- shape edges: chunked routing, large batches, the unit limit ------------------------
+
+def _random_problem(seed, B, Hkv, M, Lmax, ragged=True, sink_share=0.5):
+    """Random bf16 problem with a chosen share of sink-like groups (queries along k0)."""
+    g = torch.Generator().manual_seed(seed)
+    Hq = Hkv * M
+    q = torch.randn(B, Hq, 128, generator=g)
+    k = torch.randn(B, Hkv, Lmax, 128, generator=g)
+    v = torch.randn(B, Hkv, Lmax, 128, generator=g)
+    k0 = k[:, :, 0].clone()
+    sink = torch.rand(B, Hkv, generator=g) < sink_share
+    q = torch.where(sink.repeat_interleave(M, dim=1).unsqueeze(-1), k0.repeat_interleave(M, dim=1) * 3.0, q)
+    seq = (torch.randint(1, Lmax + 1, (B,), generator=g, dtype=torch.int32) if ragged
+           else torch.full((B,), Lmax, dtype=torch.int32))
+    bf = lambda t: t.to(torch.bfloat16)  # noqa: E731
+    kb = bf(k)
+    return inputs.DecodeInputs(inputs.WORKLOADS["tiny_4k"], seed, bf(q), kb, bf(v), kb[:, :, 0].clone(),
+                               bf(v)[:, :, 0].clone(), seq, sink, 0.6).to(DEV)
+
+
+@pytest.mark.parametrize("B,Hkv,M,Lmax", [
+    (16, 8, 8, 300),     # 128 units of M = 8: the routing kernel stages rows in two chunks
+    (4200, 1, 2, 40),    # B beyond the shared seq_lens table; 20 routing chunks
+    (16384, 1, 1, 17),   # the unit limit: prologue tables fill the whole stage area
+])
+def test_shape_edges(B, Hkv, M, Lmax):
+    x = _random_problem(40 + B, B, Hkv, M, Lmax)
+    for fused in (False, True):
+        dec = native.Decoder(B, Hkv * M, Hkv, Lmax)
+        if fused:
+            out = dec.step_fused(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+        else:
+            out = dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+        torch.cuda.synchronize()
+        assert dec.workspace.device_error() == 0
+        mr, ar, _ = oracle.route(x.q.cpu(), x.k0.cpu(), H.tau32(x.tau))
+        H.assert_route_equal(dec.route_mask.cpu(), dec.active_list.cpu(), mr, ar)
+        units = list(range(B * Hkv))
+        if len(units) > 600:  # sample: every sink plus a spread of active units
+            act = [u for u in units if mr[u] == 0]
+            units = sorted(set([u for u in units if mr[u] == 1][:300] + act[::max(1, len(act) // 300)]))
+        H.check_against_oracle(x, out.cpu(), dec.route_mask.cpu(), units=units, what=f"{B}x{Hkv}x{M}")
+
+
+def test_forced_splits_beyond_length():
+    """More forced splits than positions: most splits are empty and must weigh 0."""
+    x = _random_problem(51, 3, 4, 4, 20, ragged=True)
+    x.seq_lens[:] = torch.tensor([1, 7, 20], dtype=torch.int32, device=DEV)
+    for ns in (16, 64):
+        mask_g, _, out_g, _ = H.gpu_step(x, n_splits=ns)
+        H.check_against_oracle(x, out_g, mask_g, what=f"n_splits={ns}")
+
+
+def test_exact_cosine_tie_routes():
+    """An exact tie is a sink on both sides, each in its own precision: with
+    q = (3, 4, 0, ...) and k0 = (1, 0, ...) the kernel's fp32 cosine is fl(3/5),
+    which equals tau = 0.6f, and the oracle's fp64 cosine is exactly 0.6, which
+    equals tau = 0.6 in fp64. (Comparing the fp64 cosine with the fp32 tau would
+    not be a tie; parity workloads keep every score 0.05 away from tau.)"""
+    x = inputs.make("tiny_4k", seed=52, device=DEV, max_ctx=128)
+    k0 = torch.zeros_like(x.k0)
+    k0[0, :, 0] = 1.0
+    q = torch.zeros_like(x.q)
+    q[0, :, 0], q[0, :, 1] = 3.0, 4.0
+    q[0, 16:32] = x.q[0, 16:32]  # groups 4-7 keep random queries
+    k0[0, 4:] = x.k0[0, 4:]
+    mask, act = native.route(q, k0, 0.6)
+    mr, ar, score = oracle.route(q.cpu(), k0.cpu(), 0.6)
+    assert score[:4].tolist() == [0.6] * 4
+    H.assert_route_equal(mask.cpu(), act.cpu(), mr, ar)
+    assert mask[:4].tolist() == [1, 1, 1, 1]
+
+
+# ---- log-sum-exp output and the routing-proxy analysis ------------------------------------
+
+def test_lse_output_matches_logsumexp_and_oracle_p0():
+    x = inputs.make_graded(seed=61, batch=4, ctx=3000, device=DEV)
+    x.seq_lens[1] = 1234
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    native.route(x.q, x.k0, 0.6, dec.route_mask, dec.active_list)
+    lse = torch.full((x.batch, x.n_q_heads), -7.0, dtype=torch.float32, device=DEV)
+    native.decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, dec.active_list, dec.out,
+                            workspace=dec.workspace, lse=lse)
+    torch.cuda.synchronize()
+    mask = dec.route_mask.cpu().view(x.batch, x.n_kv_heads).repeat_interleave(4, dim=1).bool()
+    lse = lse.cpu().double()
+    assert torch.isnan(lse[mask]).all()
+    q, k = x.q.cpu().double(), x.k_cache.cpu().double()
+    for b in range(x.batch):
+        L = int(x.seq_lens[b])
+        logits = torch.einsum("hd,hld->hl", q[b], k[b].repeat_interleave(4, dim=0)[:, :L]) / math.sqrt(128)
+        ref = torch.logsumexp(logits, dim=-1)
+        act = ~mask[b]
+        assert (lse[b][act] - ref[act]).abs().max().item() < 2e-3
+    p0 = proxy_quality.full_attention_p0(x).cpu().double()
+    ref = H.oracle_full(x, float("inf")).p0
+    assert (p0 - ref).abs().max().item() < 1e-2
+
+
+def test_proxy_quality_analysis_runs_and_matches_oracle_event():
+    x = inputs.make_graded(seed=62, batch=16, ctx=2048, device=DEV)
+    res = proxy_quality.evaluate(x, taus=[0.2, 0.4, 0.55, 0.6, 0.8], cutoff=0.5)
+    assert 0.0 < res["event_rate"] < 1.0 and len(res["curve"]) == 5
+    ref = H.oracle_full(x, float("inf"))
+    ev_ref = ref.p0.view(16, 8, 4).mean(-1) >= 0.5
+    p0 = proxy_quality.full_attention_p0(x).cpu().view(16, 8, 4).mean(-1)
+    near = (p0 - 0.5).abs() < 0.02  # decisions this close to the cutoff may differ by rounding
+    assert torch.equal((p0 >= 0.5)[~near], ev_ref[~near])
