@@ -15,6 +15,8 @@ the C source:
 * ``decode`` -- sink groups return the position-0 value; active groups run
   plain softmax attention over the whole cache (README decode list; pith.science
   review of arXiv 2604.16883, Figure 1 caption, eq. (1)).
+* ``rope_append`` -- the step before: rotary embedding of the query and of the
+  new key, cache append, position-0 capture (README decode list).
 """
 from __future__ import annotations
 
@@ -59,6 +61,10 @@ class Oracle:
         self._lib.sr_oracle_decode.argtypes = [ci, ci, ci, ci, ci, u16p, u16p, u16p, u16p,
                                                i32p, u8p, i32p, ci, f64p, f64p, ci]
         self._lib.sr_oracle_decode.restype = ci
+        f32p = ctypes.POINTER(ctypes.c_float)
+        self._lib.sr_oracle_rope_append.argtypes = [ci, ci, ci, ci, ci, ci, u16p, u16p, u16p, f32p, f32p, i32p,
+                                                    u16p, u16p, u16p, u16p, u16p]
+        self._lib.sr_oracle_rope_append.restype = ci
 
     @staticmethod
     def _bits(t: torch.Tensor):
@@ -126,6 +132,36 @@ class Oracle:
         if st != 0:
             raise ValueError(f"sr_oracle_decode failed with status {st}")
         return out, p0
+
+
+def _rope_append(o: "Oracle", q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache, v_cache, k0, v0):
+    """See Oracle.rope_append."""
+    B, Hq, d = q_in.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    max_pos = rope_cos.shape[0]
+    kc = k_cache.detach().to("cpu").contiguous().clone()
+    vc = v_cache.detach().to("cpu").contiguous().clone()
+    k0c = k0.detach().to("cpu").contiguous().clone()
+    v0c = v0.detach().to("cpu").contiguous().clone()
+    sl = seq_lens.detach().to("cpu", torch.int32).contiguous().clone()
+    q_out = torch.empty((B, Hq, d), dtype=torch.bfloat16)
+    cs = rope_cos.detach().to("cpu", torch.float32).contiguous()
+    sn = rope_sin.detach().to("cpu", torch.float32).contiguous()
+    qv, qp = o._bits(q_in)
+    kv_, kp = o._bits(k_new)
+    vv_, vp = o._bits(v_new)
+    u16 = lambda t: ctypes.cast(t.view(torch.int16).data_ptr(), ctypes.POINTER(ctypes.c_uint16))  # noqa: E731
+    st = o._lib.sr_oracle_rope_append(B, Hq, Hkv, d, Lmax, max_pos, qp, kp, vp, o._ptr(cs, ctypes.c_float),
+                                      o._ptr(sn, ctypes.c_float), o._ptr(sl, ctypes.c_int32), u16(kc), u16(vc),
+                                      u16(k0c), u16(v0c), u16(q_out))
+    return st, q_out, kc, vc, k0c, v0c, sl
+
+
+Oracle.rope_append = lambda self, *a: _rope_append(self, *a)
+Oracle.rope_append.__doc__ = """The step before the scan on CPU copies: returns (status, q_out, k_cache,
+v_cache, k0, v0, seq_lens) after RoPE of q and of the new key at slot
+seq_lens[b], the append, the position-0 capture and the length update.
+status 0 = ok, 1 = some slot out of range (that sequence untouched)."""
 
 
 @dataclass

@@ -112,6 +112,96 @@ int sr_oracle_route(int B, int Hq, int Hkv, int d,
     return SR_ORACLE_OK;
 }
 
+/*
+ * Round-to-nearest-even of an fp64 value to bf16 (the top half of an IEEE
+ * fp32), in one rounding step: the value is scaled so that the bf16 spacing
+ * at its magnitude becomes 1, rounded with rint (ties to even in the default
+ * rounding mode) and scaled back; the result has at most 8 significant bits,
+ * so its conversion to fp32 is exact (or overflows to infinity).
+ */
+static uint16_t narrow_to_bf16(double x)
+{
+    if (isnan(x))
+        return 0x7fc0;
+    if (x == 0.0)
+        return signbit(x) ? 0x8000 : 0x0000;
+    int e;
+    (void)frexp(x, &e); /* |x| = m 2^e with m in [0.5, 1) */
+    int spacing = e - 8;
+    if (spacing < -133) /* bf16 subnormals share fp32's exponent range */
+        spacing = -133;
+    double y = ldexp(rint(ldexp(x, -spacing)), spacing);
+    float f = (float)y;
+    uint32_t w;
+    memcpy(&w, &f, sizeof w);
+    return (uint16_t)(w >> 16);
+}
+
+/*
+ * Rotary position embedding of one row of d values at one position
+ * (rotate-half form: element i pairs with element i + d/2):
+ *   out[i]       = x[i] c_i - x[i + d/2] s_i
+ *   out[i + d/2] = x[i + d/2] c_i + x[i] s_i,      i < d/2
+ * with c, s the rows of the cos / sin tables for that position.
+ */
+static void rope_row(const uint16_t *x, const float *c, const float *s, int d, uint16_t *out)
+{
+    int h = d / 2;
+    for (int i = 0; i < h; ++i) {
+        double a = widen_bf16(x[i]), b = widen_bf16(x[i + h]);
+        out[i] = narrow_to_bf16(a * (double)c[i] - b * (double)s[i]);
+        out[i + h] = narrow_to_bf16(b * (double)c[i] + a * (double)s[i]);
+    }
+}
+
+/*
+ * The step just before the scan, for one new token per sequence (SinkRouter
+ * README, decode-time procedure list: routing compares the RoPE query with the
+ * cached position-0 key, which prefill records; the new token's key and value
+ * join the cache). For sequence b the token takes slot p = seq_lens[b]:
+ *   q_out[b, h]  = bf16(rope(q_in[b, h], p))                for every query head
+ *   K[b, g, p]   = bf16(rope(k_new[b, g], p)),  V[b, g, p] = v_new[b, g]
+ *   k0[b, g] = K[b, g, 0], v0[b, g] = V[b, g, 0]            when p == 0
+ *   seq_lens[b] = p + 1
+ * rope_cos / rope_sin: fp32 [max_pos, d/2]. A slot outside [0, min(Lmax,
+ * max_pos)) is an error (status SR_ORACLE_BAD_ARG, nothing written for it).
+ */
+int sr_oracle_rope_append(int B, int Hq, int Hkv, int d, int Lmax, int max_pos,
+                          const uint16_t *q_in, const uint16_t *k_new, const uint16_t *v_new,
+                          const float *rope_cos, const float *rope_sin, int32_t *seq_lens,
+                          uint16_t *k_cache, uint16_t *v_cache, uint16_t *k0, uint16_t *v0, uint16_t *q_out)
+{
+    if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || d < 2 || d % 2 != 0 || Lmax < 1 || max_pos < 1 ||
+        !q_in || !k_new || !v_new || !rope_cos || !rope_sin || !seq_lens || !k_cache || !v_cache || !k0 || !v0 ||
+        !q_out)
+        return SR_ORACLE_BAD_ARG;
+    int status = SR_ORACLE_OK;
+    for (int b = 0; b < B; ++b) {
+        int p = seq_lens[b];
+        if (p < 0 || p >= Lmax || p >= max_pos) {
+            status = SR_ORACLE_BAD_ARG;
+            continue;
+        }
+        const float *c = rope_cos + (size_t)p * (d / 2);
+        const float *s = rope_sin + (size_t)p * (d / 2);
+        for (int h = 0; h < Hq; ++h)
+            rope_row(q_in + ((size_t)b * Hq + h) * d, c, s, d, q_out + ((size_t)b * Hq + h) * d);
+        for (int g = 0; g < Hkv; ++g) {
+            size_t unit = (size_t)b * Hkv + g;
+            uint16_t *kslot = k_cache + (unit * Lmax + p) * d;
+            uint16_t *vslot = v_cache + (unit * Lmax + p) * d;
+            rope_row(k_new + unit * d, c, s, d, kslot);
+            memcpy(vslot, v_new + unit * d, sizeof(uint16_t) * (size_t)d);
+            if (p == 0) {
+                memcpy(k0 + unit * d, kslot, sizeof(uint16_t) * (size_t)d);
+                memcpy(v0 + unit * d, vslot, sizeof(uint16_t) * (size_t)d);
+            }
+        }
+        seq_lens[b] = p + 1;
+    }
+    return status;
+}
+
 typedef struct {
     int B, Hq, Hkv, d, Lmax;
     const uint16_t *q, *kc, *vc, *v0;

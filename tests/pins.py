@@ -276,6 +276,101 @@ def pin_active_list_order(o):
     assert mask.view(5, 8).bool().equal(pick)
 
 
+# --- the step before the scan: RoPE, append, position-0 capture ----------------------
+
+def _rope_case(seed, B, Hkv, M, Lmax, max_pos=64, d=128):
+    g = torch.Generator().manual_seed(seed)
+    Hq = Hkv * M
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    k0 = kc[:, :, 0].clone()
+    v0 = vc[:, :, 0].clone()
+    inv = 500000.0 ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * inv[None, :]
+    return q, kn, vn, kc, vc, k0, v0, torch.cos(ang).float(), torch.sin(ang).float()
+
+
+def pin_rope_identity_at_position_zero(o):
+    """At position 0 (cos 1, sin 0) the rotation is the identity: the query is
+    unchanged, the new key / value land in slot 0 and become k0 / v0."""
+    q, kn, vn, kc, vc, k0, v0, cs, sn = _rope_case(81, 2, 3, 4, 16)
+    seq = torch.zeros(2, dtype=torch.int32)
+    st, qo, kc2, vc2, k02, v02, sl = o.rope_append(q, kn, vn, cs, sn, seq, kc, vc, k0, v0)
+    assert st == 0 and sl.tolist() == [1, 1]
+    assert torch.equal(qo.view(torch.int16), q.view(torch.int16))
+    assert torch.equal(kc2[:, :, 0].view(torch.int16), kn.view(torch.int16))
+    assert torch.equal(vc2[:, :, 0].view(torch.int16), vn.view(torch.int16))
+    assert torch.equal(k02.view(torch.int16), kn.view(torch.int16))
+    assert torch.equal(v02.view(torch.int16), vn.view(torch.int16))
+    assert torch.equal(kc2[:, :, 1:], kc[:, :, 1:])
+
+
+def pin_rope_closed_form_and_ties(o):
+    """Exact values: x_i = 2, x_(i+64) = 1 with c = 0.5, s = 0.75 gives
+    (2*0.5 - 1*0.75, 1*0.5 + 2*0.75) = (0.25, 2). Ties round to even:
+    1 + 2^-8 (between 1 and 1 + 2^-7) -> 1, and 1 + 3*2^-8 -> 1 + 2^-6."""
+    d = 128
+    q = torch.zeros(1, 3, d, dtype=torch.bfloat16)
+    q[0, 0, 5], q[0, 0, 69] = 2.0, 1.0
+    q[0, 1, 7] = 1.0
+    q[0, 2, 9] = 1.0
+    cs = torch.zeros(4, 64)
+    sn = torch.zeros(4, 64)
+    cs[3, 5], sn[3, 5] = 0.5, 0.75
+    cs[3, 7] = 1.0 + 2.0 ** -8
+    cs[3, 9] = 1.0 + 3 * 2.0 ** -8
+    kc = torch.zeros(1, 1, 8, d, dtype=torch.bfloat16)
+    st, qo, *_ = o.rope_append(q.view(1, 3, d), torch.zeros(1, 1, d, dtype=torch.bfloat16),
+                               torch.zeros(1, 1, d, dtype=torch.bfloat16), cs, sn,
+                               torch.tensor([3], dtype=torch.int32), kc, kc.clone(),
+                               torch.zeros(1, 1, d, dtype=torch.bfloat16), torch.zeros(1, 1, d, dtype=torch.bfloat16))
+    assert st == 0
+    assert qo[0, 0, 5].item() == 0.25 and qo[0, 0, 69].item() == 2.0
+    assert qo[0, 1, 7].item() == 1.0
+    assert qo[0, 2, 9].item() == 1.0 + 2.0 ** -6
+
+
+def pin_rope_rotation_preserves_norm_and_inverts(o):
+    """A true rotation keeps every pair's norm (up to bf16 rounding), and
+    rotating by an angle then by its negative returns the input."""
+    q, kn, vn, kc, vc, k0, v0, cs, sn = _rope_case(82, 2, 2, 2, 48, max_pos=64)
+    seq = torch.tensor([17, 40], dtype=torch.int32)
+    st, qo, *_ = o.rope_append(q, kn, vn, cs, sn, seq, kc, vc, k0, v0)
+    assert st == 0
+    a, b = q.double()[..., :64], q.double()[..., 64:]
+    c, d_ = qo.double()[..., :64], qo.double()[..., 64:]
+    n_in, n_out = (a * a + b * b).sqrt(), (c * c + d_ * d_).sqrt()
+    assert ((n_out - n_in).abs() <= 2.0 ** -7 * n_in + 1e-30).all()
+    # inverse: a table whose row p holds the negative angle
+    sn_neg = -sn
+    st2, back, *_ = o.rope_append(qo, kn, vn, cs, sn_neg, seq, kc, vc, k0, v0)
+    assert st2 == 0
+    # two bf16 roundings of a rotated pair, each at most 2^-9 of the pair's norm
+    err = (back.double() - q.double()).abs()
+    assert (err[..., :64] <= 2.0 ** -7 * n_in).all() and (err[..., 64:] <= 2.0 ** -7 * n_in).all()
+
+
+def pin_rope_append_bookkeeping(o):
+    """Only slot p is written, k0 / v0 change only when p == 0, lengths advance,
+    and a slot past the cache or the table is refused for that sequence."""
+    q, kn, vn, kc, vc, k0, v0, cs, sn = _rope_case(83, 3, 2, 2, 10, max_pos=64)
+    seq = torch.tensor([4, 0, 10], dtype=torch.int32)  # the last one is full
+    st, qo, kc2, vc2, k02, v02, sl = o.rope_append(q, kn, vn, cs, sn, seq, kc, vc, k0, v0)
+    assert st == 1 and sl.tolist() == [5, 1, 10]
+    for b, p in ((0, 4), (1, 0)):
+        keep = [j for j in range(10) if j != p]
+        assert torch.equal(kc2[b][:, keep], kc[b][:, keep]) and torch.equal(vc2[b][:, keep], vc[b][:, keep])
+        assert torch.equal(vc2[b, :, p].view(torch.int16), vn[b].view(torch.int16))
+    assert torch.equal(k02[0], k0[0]) and torch.equal(v02[0], v0[0])  # p = 4: k0 kept
+    assert torch.equal(k02[1], kc2[1, :, 0]) and torch.equal(v02[1], vn[1])  # p = 0: captured
+    assert torch.equal(kc2[2], kc[2]) and torch.equal(k02[2], k0[2])  # refused: untouched
+
+
 PINS = [pin_dense_matches_sdpa, pin_all_sinks_return_v0, pin_routing_isolation,
         pin_planted_sink_bound, pin_permutation_invariance, pin_closed_forms,
-        pin_hand_worked, pin_route_geometry, pin_route_scale_invariance, pin_active_list_order]
+        pin_hand_worked, pin_route_geometry, pin_route_scale_invariance, pin_active_list_order,
+        pin_rope_identity_at_position_zero, pin_rope_closed_form_and_ties,
+        pin_rope_rotation_preserves_norm_and_inverts, pin_rope_append_bookkeeping]

@@ -29,6 +29,16 @@ MUTANTS = [
      "const uint16_t *v0g = V + (size_t)d;"),
     ("p0_reports_last_weight", "J->p0[(size_t)b * J->Hq + h] = logit[0] / z;",
      "J->p0[(size_t)b * J->Hq + h] = logit[L - 1] / z;"),
+    ("rope_sign", "out[i] = narrow_to_bf16(a * (double)c[i] - b * (double)s[i]);",
+     "out[i] = narrow_to_bf16(a * (double)c[i] + b * (double)s[i]);"),
+    ("rope_adjacent_pairs", "double a = widen_bf16(x[i]), b = widen_bf16(x[i + h]);",
+     "double a = widen_bf16(x[i]), b = widen_bf16(x[(i + 1) % d]);"),
+    ("no_position0_capture", "memcpy(k0 + unit * d, kslot, sizeof(uint16_t) * (size_t)d);", ""),
+    ("length_not_advanced", "seq_lens[b] = p + 1;", "seq_lens[b] = p;"),
+    ("ties_away_from_zero", "double y = ldexp(rint(ldexp(x, -spacing)), spacing);",
+     "double y = ldexp(round(ldexp(x, -spacing)), spacing);"),
+    ("rope_row_of_next_position", "const float *c = rope_cos + (size_t)p * (d / 2);",
+     "const float *c = rope_cos + (size_t)(p + 1) * (d / 2);"),
 ]
 
 
