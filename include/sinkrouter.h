@@ -65,6 +65,8 @@ typedef enum sr_status {
 #define SR_DEVERR_TIMEOUT 4     /* a pipeline wait exceeded its time bound (a bug, never
                                    expected); outputs of that launch are invalid and the
                                    workspace must be re-initialised with sr_workspace_init */
+#define SR_DEVERR_APPEND_SLOT 8 /* sr_rope_append_route: a sequence's slot seq_lens[b] was
+                                   outside [0, min(Lmax, max_pos)); nothing was appended for it */
 
 /*
  * sr_route -- cosine routing of every unit (README decode list: compare the RoPE
@@ -89,6 +91,53 @@ typedef enum sr_status {
  */
 sr_status sr_route(const sr_dims *dims, const void *q, const void *k0, float tau,
                    uint8_t *route_mask, int32_t *active_list, void *stream);
+
+/*
+ * sr_rope_append_route -- the step just before the scan, in one launch, for one
+ * new token per sequence (README decode list: routing compares the RoPE'd query
+ * with the cached position-0 key, which is recorded when the first token is
+ * written; the new token's key and value join the cache before the scan). For
+ * sequence b the token takes slot p = seq_lens[b]:
+ *     q_out[b, h]   = rope(q_in[b, h], p)                  every query head h
+ *     K[b, g, p]    = rope(k_new[b, g], p);   V[b, g, p] = v_new[b, g]
+ *     k0[b, g] = K[b, g, 0], v0[b, g] = V[b, g, 0]          when p == 0
+ *     route_mask / active_list = sr_route(q_out, k0, tau)  (bit for bit)
+ *     seq_lens[b]   = p + 1
+ * rope is the rotate-half rotary embedding: for i < d/2, with c = cos[p, i],
+ * s = sin[p, i],
+ *     y[i] = x[i] c - x[i + d/2] s,    y[i + d/2] = x[i + d/2] c + x[i] s,
+ * each element the correctly rounded bf16 (nearest, ties to even) of that
+ * value computed from the bf16 x and the fp32 table entries. The tables are
+ * the caller's, so any frequency schedule (base, scaling) can be used.
+ *
+ *   q_in        bf16 [B, Hq, d]   query before RoPE (may be the same buffer as
+ *                                 q_out: rotated in place)
+ *   k_new       bf16 [B, Hkv, d]  new key before RoPE; must not overlap the caches
+ *   v_new       bf16 [B, Hkv, d]  new value; must not overlap the caches
+ *   rope_cos    fp32 [max_pos, d/2] cos table, row p for position p
+ *   rope_sin    fp32 [max_pos, d/2] sin table
+ *   max_pos     rows of the tables (>= 1)
+ *   seq_lens    in/out int32 [B]: the slot to write, advanced by one
+ *   k_cache, v_cache  in/out bf16 [B, Hkv, Lmax, d]: slot p is written
+ *   k0, v0      in/out bf16 [B, Hkv, d]: written when p == 0, else read (k0)
+ *   tau         routing threshold, as for sr_route
+ *   q_out       out bf16 [B, Hq, d]: the RoPE'd query sr_decode_attention takes
+ *   route_mask, active_list  out, as for sr_route
+ *   device_error optional device int32 (NULL = not wanted): SR_DEVERR_APPEND_SLOT
+ *               is ORed in when a sequence's slot is outside [0, min(Lmax,
+ *               max_pos)) -- its cache, k0/v0 and length are left untouched,
+ *               its q_out rows are zero and its groups are routed from those
+ *               rows (so the mask still equals sr_route(q_out, k0, tau))
+ * One launch of one CTA; no workspace. It waits for the preceding kernel in the
+ * stream before reading anything and lets the next one (sr_decode_attention,
+ * which reads all of its inputs after its own wait) launch early. Errors:
+ * SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_CUDA.
+ */
+sr_status sr_rope_append_route(const sr_dims *dims, const void *q_in, const void *k_new,
+                               const void *v_new, const float *rope_cos, const float *rope_sin,
+                               int32_t max_pos, int32_t *seq_lens, void *k_cache, void *v_cache,
+                               void *k0, void *v0, float tau, void *q_out, uint8_t *route_mask,
+                               int32_t *active_list, int32_t *device_error, void *stream);
 
 /*
  * sr_decode_workspace_bytes -- size of the workspace sr_decode_attention needs

@@ -83,6 +83,49 @@ sr_status sr_route(const sr_dims *dims, const void *q, const void *k0, float tau
     return e == cudaSuccess ? SR_OK : cuda_fail(e);
 }
 
+sr_status sr_rope_append_route(const sr_dims *dims, const void *q_in, const void *k_new, const void *v_new,
+                               const float *rope_cos, const float *rope_sin, int32_t max_pos, int32_t *seq_lens,
+                               void *k_cache, void *v_cache, void *k0, void *v0, float tau, void *q_out,
+                               uint8_t *route_mask, int32_t *active_list, int32_t *device_error, void *stream)
+{
+    const sr_status st = check_dims(dims);
+    if (st != SR_OK)
+        return st;
+    const void *rows[] = {q_in, k_new, v_new, rope_cos, rope_sin, k_cache, v_cache, k0, v0, q_out};
+    for (const void *r : rows)
+        if (!r || !aligned(r, 16))
+            return SR_ERR_INVALID_ARG;
+    if (!seq_lens || !aligned(seq_lens, 4) || !route_mask || !active_list || !aligned(active_list, 4))
+        return SR_ERR_INVALID_ARG;
+    if (device_error && !aligned(device_error, 4))
+        return SR_ERR_INVALID_ARG;
+    if (max_pos < 1 || std::isnan(tau))
+        return SR_ERR_INVALID_ARG;
+    sr::PrestepArgs a;
+    a.q_in = q_in;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.rope_cos = rope_cos;
+    a.rope_sin = rope_sin;
+    a.seq_lens = seq_lens;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.k0 = k0;
+    a.v0 = v0;
+    a.q_out = q_out;
+    a.mask = route_mask;
+    a.active = active_list;
+    a.error = device_error;
+    a.tau = tau;
+    a.batch = dims->batch;
+    a.n_q_heads = dims->n_q_heads;
+    a.n_kv_heads = dims->n_kv_heads;
+    a.max_seq_len = dims->max_seq_len;
+    a.max_pos = max_pos;
+    const cudaError_t e = sr::launch_rope_append_route(a, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
 size_t sr_decode_workspace_bytes(const sr_dims *dims, int32_t max_splits)
 {
     if (check_dims(dims) != SR_OK || max_splits < 0 || max_splits > SR_MAX_SPLITS)

@@ -284,17 +284,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     int n = 0;
     long long local = 0;
     if constexpr (!FUSED) {
-        // seq_lens is a caller input that was complete before the routing
-        // kernel ran, so it is staged before the dependency wait; the active
-        // list is the routing kernel's output and is read only after it.
-        if (seq_smem)
-            for (int b = tid; b < p.B; b += kThreads)
-                seqtab[b] = __ldg(p.seq_lens + b);
+        // The preceding kernel may have written every input (the routing
+        // kernel writes the active list; the append step also advances
+        // seq_lens), so all of them are read after the dependency wait, the
+        // length table and the list count in the same round trip.
         grid_dependency_wait();
         grid_launch_dependents();
         __syncthreads();
 
         n = __ldg(p.active);
+        if (seq_smem)
+            for (int b = tid; b < p.B; b += kThreads)
+                seqtab[b] = __ldg(p.seq_lens + b);
         if (n < 0 || n > U) {
             errbits |= SR_DEVERR_ACTIVE_LIST;
             n = n < 0 ? 0 : U;

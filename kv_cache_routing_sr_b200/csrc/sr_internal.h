@@ -69,7 +69,21 @@ struct DecodeArgs {
     float *lse = nullptr;
 };
 
+// RoPE + append + position-0 capture + routing (sr_rope_append_route).
+struct PrestepArgs {
+    const void *q_in, *k_new, *v_new;
+    const float *rope_cos, *rope_sin;
+    int32_t *seq_lens;
+    void *k_cache, *v_cache, *k0, *v0, *q_out;
+    uint8_t *mask;
+    int32_t *active;
+    int32_t *error;
+    float tau;
+    int batch, n_q_heads, n_kv_heads, max_seq_len, max_pos;
+};
+
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);
+cudaError_t launch_rope_append_route(const PrestepArgs &a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 // Persistent CTAs of the decode kernel on the current device (0 on error).
 int decode_grid_size();

@@ -51,7 +51,6 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
     __shared__ int32_t warp_off[kRouteWarps + 1];
 
     const int U = B * Hkv;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint4 *rows = reinterpret_cast<uint4 *>(dsm);
     uint8_t *sink_flag = dsm + (size_t)cu * (M + 1) * 256;
     const uint32_t b = smem_u32(&bar);
@@ -101,38 +100,7 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
         return;
     }
 
-    // Ordered compaction of the active units.
-    int32_t total = 0;
-    for (int c0 = 0; c0 < U; c0 += kRouteThreads) {
-        const int u = c0 + (int)threadIdx.x;
-        const bool act = (u < U) && !sink_flag[u];
-        const unsigned ball = __ballot_sync(0xffffffffu, act);
-        const int before = __popc(ball & ((1u << lane) - 1u));
-        if (lane == 0)
-            warp_cnt[warp] = __popc(ball);
-        __syncthreads();
-        if (warp == 0) {
-            const int v = (lane < kRouteWarps) ? warp_cnt[lane] : 0;
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o)
-                    incl += y;
-            }
-            if (lane < kRouteWarps)
-                warp_off[lane] = incl - v;
-            if (lane == kRouteWarps - 1)
-                warp_off[kRouteWarps] = incl;
-        }
-        __syncthreads();
-        if (act)
-            active[1 + total + warp_off[warp] + before] = u;
-        total += warp_off[kRouteWarps];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0)
-        active[0] = total;
+    compact_active<kRouteThreads>(sink_flag, U, active, warp_cnt, warp_off);
 }
 
 template <int M>

@@ -1,6 +1,7 @@
-// Cosine of one query head with its group's position-0 key, shared by the
-// routing kernel and the fused route + decode prologue so that both take the
-// same decision bit for bit.
+// Cosine of one query head with its group's position-0 key and the ordered
+// compaction of the active units, shared by the routing kernel, the fused
+// route + decode prologue and the RoPE + append + route step, so that all of
+// them take the same decision bit for bit.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -126,6 +127,54 @@ __device__ __forceinline__ void route_staged(const uint4 *rows, int u0, int nu, 
                 mask_out[u0 + lu] = sink;
         }
     }
+}
+
+} // namespace sr
+
+namespace sr {
+
+// Ordered compaction: active[0] = number of units u < U with sflag[u] == 0,
+// active[1..] = those units in ascending order. Warp ballots give each lane's
+// rank inside its warp and a one-warp scan of the per-warp counts gives the
+// warp offsets, NT threads at a time. Called by all NT threads of the block;
+// warp_cnt / warp_off are shared arrays of NT/32 and NT/32 + 1 entries.
+template <int NT>
+__device__ __forceinline__ void compact_active(const uint8_t *sflag, int U, int32_t *active, int32_t *warp_cnt,
+                                               int32_t *warp_off)
+{
+    constexpr int kWarps = NT / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t total = 0;
+    for (int c0 = 0; c0 < U; c0 += NT) {
+        const int u = c0 + (int)threadIdx.x;
+        const bool act = (u < U) && !sflag[u];
+        const unsigned ball = __ballot_sync(0xffffffffu, act);
+        const int before = __popc(ball & ((1u << lane) - 1u));
+        if (lane == 0)
+            warp_cnt[warp] = __popc(ball);
+        __syncthreads();
+        if (warp == 0) {
+            const int v = (lane < kWarps) ? warp_cnt[lane] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += y;
+            }
+            if (lane < kWarps)
+                warp_off[lane] = incl - v;
+            if (lane == kWarps - 1)
+                warp_off[kWarps] = incl;
+        }
+        __syncthreads();
+        if (act)
+            active[1 + total + warp_off[warp] + before] = u;
+        total += warp_off[kWarps];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        active[0] = total;
 }
 
 } // namespace sr

@@ -33,7 +33,8 @@ IMAGE_TOKENS = 576
 IMAGE_SCALE = 1.5
 
 # Seed offsets per tensor role, so each role has its own stream.
-_ROLE = {"k": 1, "v": 2, "k0dir": 3, "qnoise": 4, "qactive": 5, "lens": 6, "sinks": 7, "strength": 8}
+_ROLE = {"k": 1, "v": 2, "k0dir": 3, "qnoise": 4, "qactive": 5, "lens": 6, "sinks": 7, "strength": 8,
+         "qin": 9, "knew": 10, "vnew": 11}
 
 
 @dataclass(frozen=True)
@@ -241,6 +242,30 @@ def make_graded(seed: int = 0, device="cpu", *, batch: int = 16, n_kv_heads: int
     w = Workload("graded", B, ctx, Hkv, M, tau=tau, description="graded sink strength t ~ U(0,1) per unit")
     return DecodeInputs(w, seed, q.to(torch.bfloat16), k_cache, v_cache, k_cache[:, :, 0].clone(),
                         v_cache[:, :, 0].clone(), seq_lens, t > 0.5, tau, extra={"strength": t})
+
+
+def rope_tables(max_pos: int, head_dim: int = HEAD_DIM, base: float = 500000.0, device="cpu"):
+    """cos / sin tables, fp32 [max_pos, head_dim / 2], for the rotate-half
+    rotary embedding: row p, column i holds cos / sin of p * base^(-2i/d).
+    base 500000 is Llama 3's; no context-extension rescaling of the frequencies
+    (synthetic inputs). The angles are formed in fp64 and the results rounded
+    to fp32. These are inputs: both the oracle and the CUDA path read them."""
+    inv = base ** (-torch.arange(0, head_dim, 2, dtype=torch.float64) / head_dim)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * inv[None, :]
+    return torch.cos(ang).float().to(device), torch.sin(ang).float().to(device)
+
+
+def make_projections(batch: int, n_q_heads: int, n_kv_heads: int, seed: int = 0, device="cpu"):
+    """The new token's projections before RoPE: q_in [B, Hq, d], k_new and
+    v_new [B, Hkv, d], N(0, 1) rounded to bf16."""
+    device = torch.device(device)
+    d = HEAD_DIM
+
+    def draw(shape, role):
+        return torch.randn(shape, generator=_gen(seed, role, device), device=device).to(torch.bfloat16)
+
+    return (draw((batch, n_q_heads, d), "qin"), draw((batch, n_kv_heads, d), "knew"),
+            draw((batch, n_kv_heads, d), "vnew"))
 
 
 def needed_bytes(seq_lens, active_units, n_kv_heads: int, n_q_heads: int, batch: int,

@@ -41,7 +41,7 @@ _lib = None
 EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_decode_attention",
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
            "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention",
-           "sr_decode_attention_lse"]
+           "sr_decode_attention_lse", "sr_rope_append_route"]
 
 
 def load(path: str = LIBRARY):
@@ -80,6 +80,9 @@ def load(path: str = LIBRARY):
     lib.sr_route_decode_attention.restype = ctypes.c_int
     lib.sr_decode_attention_lse.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, u64, vp]
     lib.sr_decode_attention_lse.restype = ctypes.c_int
+    lib.sr_rope_append_route.argtypes = [dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                         vp, vp, vp]
+    lib.sr_rope_append_route.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -227,6 +230,37 @@ def route_decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, tau, out=None,
     return out
 
 
+def rope_append_route(q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache, v_cache, k0, v0, tau,
+                      q_out=None, route_mask=None, active_list=None, device_error=None, stream=None):
+    """sr_rope_append_route: RoPE of the query and the new key at slot
+    seq_lens[b], append of the new key / value, position-0 capture, routing and
+    the length update, in one launch. Updates k_cache, v_cache, k0, v0 and
+    seq_lens in place; returns (q_out, route_mask, active_list). q_out may be
+    q_in (rotated in place)."""
+    B, Hq, d = q_in.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if q_out is None:
+        q_out = torch.empty_like(q_in)
+    if route_mask is None:
+        route_mask = torch.empty(B * Hkv, dtype=torch.uint8, device=q_in.device)
+    if active_list is None:
+        active_list = torch.empty(1 + B * Hkv, dtype=torch.int32, device=q_in.device)
+    if rope_cos.shape != rope_sin.shape or rope_cos.dim() != 2 or rope_cos.shape[1] != d // 2:
+        raise ValueError("rope_cos / rope_sin must both be [max_pos, head_dim / 2]")
+    err = 0 if device_error is None else _dev(device_error, "device_error", torch.int32)
+    dims = dims_of(B, Hq, Hkv, Lmax, d)
+    st = load().sr_rope_append_route(
+        ctypes.byref(dims), _dev(q_in, "q_in", torch.bfloat16), _dev(k_new, "k_new", torch.bfloat16),
+        _dev(v_new, "v_new", torch.bfloat16), _dev(rope_cos, "rope_cos", torch.float32),
+        _dev(rope_sin, "rope_sin", torch.float32), int(rope_cos.shape[0]), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(k0, "k0", torch.bfloat16), _dev(v0, "v0", torch.bfloat16), float(tau),
+        _dev(q_out, "q_out", torch.bfloat16), _dev(route_mask, "route_mask", torch.uint8),
+        _dev(active_list, "active_list", torch.int32), err or None, _stream(stream))
+    _check("sr_rope_append_route", st)
+    return q_out, route_mask, active_list
+
+
 def grid_size() -> int:
     return int(load().sr_decode_grid_size())
 
@@ -247,6 +281,20 @@ class Decoder:
     def step(self, q, k_cache, v_cache, k0, v0, seq_lens, tau, n_splits: int = 0, stream=None):
         route(q, k0, tau, self.route_mask, self.active_list, stream)
         decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, self.active_list, self.out, n_splits,
+                         self.workspace, stream)
+        return self.out
+
+    def append_step(self, q_in, k_new, v_new, rope_cos, rope_sin, k_cache, v_cache, k0, v0, seq_lens, tau,
+                    n_splits: int = 0, device_error=None, stream=None):
+        """A whole decode step from the un-rotated projections:
+        sr_rope_append_route (RoPE, append, capture, route, lengths) then
+        sr_decode_attention on the rotated query. The caches, k0 / v0 and
+        seq_lens are updated in place; the rotated query is kept in self.q."""
+        if getattr(self, "q", None) is None or self.q.shape != q_in.shape:
+            self.q = torch.empty_like(q_in)
+        rope_append_route(q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache, v_cache, k0, v0, tau,
+                          self.q, self.route_mask, self.active_list, device_error, stream)
+        decode_attention(self.q, k_cache, v_cache, k0, v0, seq_lens, self.active_list, self.out, n_splits,
                          self.workspace, stream)
         return self.out
 

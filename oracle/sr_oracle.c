@@ -164,7 +164,9 @@ static void rope_row(const uint16_t *x, const float *c, const float *s, int d, u
  *   k0[b, g] = K[b, g, 0], v0[b, g] = V[b, g, 0]            when p == 0
  *   seq_lens[b] = p + 1
  * rope_cos / rope_sin: fp32 [max_pos, d/2]. A slot outside [0, min(Lmax,
- * max_pos)) is an error (status SR_ORACLE_BAD_ARG, nothing written for it).
+ * max_pos)) is an error (status SR_ORACLE_BAD_ARG): that sequence's cache,
+ * k0/v0 and length are left alone and its q_out rows are zero (there is no
+ * table row to rotate by; the pages do not cover a full cache).
  */
 int sr_oracle_rope_append(int B, int Hq, int Hkv, int d, int Lmax, int max_pos,
                           const uint16_t *q_in, const uint16_t *k_new, const uint16_t *v_new,
@@ -180,6 +182,7 @@ int sr_oracle_rope_append(int B, int Hq, int Hkv, int d, int Lmax, int max_pos,
         int p = seq_lens[b];
         if (p < 0 || p >= Lmax || p >= max_pos) {
             status = SR_ORACLE_BAD_ARG;
+            memset(q_out + (size_t)b * Hq * d, 0, sizeof(uint16_t) * (size_t)Hq * d);
             continue;
         }
         const float *c = rope_cos + (size_t)p * (d / 2);

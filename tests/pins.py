@@ -367,6 +367,7 @@ def pin_rope_append_bookkeeping(o):
     assert torch.equal(k02[0], k0[0]) and torch.equal(v02[0], v0[0])  # p = 4: k0 kept
     assert torch.equal(k02[1], kc2[1, :, 0]) and torch.equal(v02[1], vn[1])  # p = 0: captured
     assert torch.equal(kc2[2], kc[2]) and torch.equal(k02[2], k0[2])  # refused: untouched
+    assert (qo[2].float() == 0).all() and (qo[:2].float() != 0).any()  # ... and a zero query
 
 
 PINS = [pin_dense_matches_sdpa, pin_all_sinks_return_v0, pin_routing_isolation,

@@ -125,3 +125,26 @@ def test_fused_entry_validation(lib):
     bad = dims(d=96)
     assert lib.sr_route_decode_attention(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.6),
                                          0, None, None, FAKE, FAKE, 1 << 30, None) == native.SR_ERR_UNSUPPORTED
+
+
+def test_rope_append_route_validation(lib):
+    """Host-side refusals of sr_rope_append_route: nothing is launched."""
+    d = dims()
+
+    def c(**kw):
+        a = dict(q_in=FAKE, k_new=FAKE, v_new=FAKE, cos=FAKE, sin=FAKE, max_pos=64, seq=FAKE, kc=FAKE, vc=FAKE,
+                 k0=FAKE, v0=FAKE, tau=0.6, q_out=FAKE, mask=FAKE, act=FAKE, err=None, dims=d)
+        a.update(kw)
+        return lib.sr_rope_append_route(ctypes.byref(a["dims"]), a["q_in"], a["k_new"], a["v_new"], a["cos"],
+                                        a["sin"], a["max_pos"], a["seq"], a["kc"], a["vc"], a["k0"], a["v0"],
+                                        ctypes.c_float(a["tau"]), a["q_out"], a["mask"], a["act"], a["err"], None)
+
+    for name in ("q_in", "k_new", "v_new", "cos", "sin", "seq", "kc", "vc", "k0", "v0", "q_out", "mask", "act"):
+        assert c(**{name: None}) == native.SR_ERR_INVALID_ARG, name
+    for name in ("q_in", "k_new", "v_new", "cos", "sin", "kc", "vc", "k0", "v0", "q_out"):
+        assert c(**{name: FAKE + 8}) == native.SR_ERR_INVALID_ARG, name  # 16-byte rows
+    assert c(seq=FAKE + 2) == native.SR_ERR_INVALID_ARG
+    assert c(err=FAKE + 2) == native.SR_ERR_INVALID_ARG
+    assert c(max_pos=0) == native.SR_ERR_INVALID_ARG
+    assert c(tau=float("nan")) == native.SR_ERR_INVALID_ARG
+    assert c(dims=dims(d=64)) == native.SR_ERR_UNSUPPORTED
