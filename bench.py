@@ -273,6 +273,89 @@ def time_kernels(native, dec, x, tau, steps, flush):
     return [e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev]
 
 
+class AppendInputs:
+    """Inputs of the decode step that starts from the un-rotated projections
+    (sr_rope_append_route then sr_decode_attention) on workload x: every
+    sequence's last cache slot takes the new token, so after the append the
+    scan covers the workload's full context. q_in is the workload's planted
+    query rotated back to that slot (by the library's own kernel, with the sine
+    table negated), so routing sees the same groups as the two-call step.
+    Each timed step restores seq_lens from seq_saved before its start event."""
+
+    def __init__(self, native, inputs, x):
+        import torch
+        dev = x.q.device
+        B, Hq, Hkv = x.batch, x.n_q_heads, x.n_kv_heads
+        self.seq_saved = (x.seq_lens - 1).clone()
+        self.seq_lens = self.seq_saved.clone()
+        self.cos, self.sin = inputs.rope_tables(x.max_seq_len, device=dev)
+        _, self.k_new, self.v_new = inputs.make_projections(B, Hq, Hkv, seed=x.seed + 17, device=dev)
+        # rotate the planted query back: one call per distinct slot, on
+        # one-slot scratch caches, with a one-row table (row p, sines negated)
+        self.q_in = torch.empty_like(x.q)
+        z1 = torch.zeros((1, Hkv, 1, 128), dtype=torch.bfloat16, device=dev)
+        for b, p in enumerate(self.seq_saved.tolist()):
+            zr = torch.zeros((1, Hkv, 128), dtype=torch.bfloat16, device=dev)
+            native.rope_append_route(x.q[b:b + 1].contiguous(), zr, zr.clone(), self.cos[p:p + 1].contiguous(),
+                                     (-self.sin[p:p + 1]).contiguous(), torch.zeros(1, dtype=torch.int32, device=dev),
+                                     z1.clone(), z1.clone(), zr.clone(), zr.clone(), float("inf"),
+                                     q_out=self.q_in[b:b + 1])
+        torch.cuda.synchronize()
+
+    def step(self, native, dec, x, tau):
+        self.seq_lens.copy_(self.seq_saved)
+        return dec.append_step(self.q_in, self.k_new, self.v_new, self.cos, self.sin, x.k_cache, x.v_cache, x.k0,
+                               x.v0, self.seq_lens, tau)
+
+
+def _captured_append_steps(native, dec, x, a, tau, steps, flush, split_events):
+    """As _captured_steps for the append path: per step an L2 flush and the
+    seq_lens reset, then an event, sr_rope_append_route, (an event,)
+    sr_decode_attention, an event."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    side = torch.cuda.Stream(device=x.q.device)
+    side.wait_stream(torch.cuda.current_stream(x.q.device))
+    with torch.cuda.stream(side):
+        a.step(native, dec, x, tau)
+        flush.sum()
+    torch.cuda.current_stream(x.q.device).wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = torch.cuda.current_stream()
+        for i in range(steps):
+            flush.sum()
+            a.seq_lens.copy_(a.seq_saved)
+            ev[i][0].record(st)
+            native.rope_append_route(a.q_in, a.k_new, a.v_new, a.cos, a.sin, a.seq_lens, x.k_cache, x.v_cache,
+                                     x.k0, x.v0, tau, dec.q, dec.route_mask, dec.active_list)
+            if split_events:
+                ev[i][1].record(st)
+            native.decode_attention(dec.q, x.k_cache, x.v_cache, x.k0, x.v0, a.seq_lens, dec.active_list, dec.out,
+                                    0, dec.workspace)
+            ev[i][2].record(st)
+    return g, ev
+
+
+def time_append(native, dec, x, a, steps, warmup):
+    """(step times, prestep kernel times) in ms of the append path."""
+    import torch
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=x.q.device)
+    gw, _ = _captured_append_steps(native, dec, x, a, x.tau, warmup, flush, False)
+    g, ev = _captured_append_steps(native, dec, x, a, x.tau, steps, flush, False)
+    gk, evk = _captured_append_steps(native, dec, x, a, x.tau, steps, flush, True)
+    gw.replay()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    steps_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    gk.replay()
+    torch.cuda.synchronize()
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evk]
+    del flush
+    return steps_ms, pre_ms
+
+
 def measure_workload(native, inputs, x, steps, warmup, flush, barrier, fused=True):
     """Timings of one workload on this GPU: the two-call step (routed and with
     routing disabled) and its kernels, and, if asked, the fused step."""
@@ -335,6 +418,44 @@ def e2e_measure(native, x, steps):
     ms = e0.elapsed_time(e1) / steps
     del dev, host
     return ms, h2d, d2h
+
+
+def e2e_append_measure(native, x, a, steps):
+    """The serving view of the same step through the public API: per step only
+    the new token's projections (q_in, k_new, v_new) come from pinned host
+    memory, the append step and the scan run against the resident cache, and
+    the output and route mask go back to the host, all inside the timed region.
+    seq_lens is restored on the device each step so that the context stays at
+    the workload's length."""
+    import torch
+    host = {n: getattr(a, n).cpu().pin_memory() for n in ("q_in", "k_new", "v_new")}
+    dev = {n: torch.empty_like(getattr(a, n)) for n in host}
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
+    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    mask_h = torch.empty(dec.route_mask.shape, dtype=dec.route_mask.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + mask_h.numel()
+    st = torch.cuda.current_stream()
+
+    def one():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        a.seq_lens.copy_(a.seq_saved)
+        dec.append_step(dev["q_in"], dev["k_new"], dev["v_new"], a.cos, a.sin, x.k_cache, x.v_cache, x.k0, x.v0,
+                        a.seq_lens, x.tau)
+        out_h.copy_(dec.out, non_blocking=True)
+        mask_h.copy_(dec.route_mask, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
 def oracle_layer_step_us(x_cpu, budget_s, min_reps=1):
@@ -433,7 +554,6 @@ def run_ours(args):
                      "kernel": "decode_kernel<1,4> (persistent split-K scan + sink copy + merge)",
                      "algorithmic_bytes_per_launch": need, "peak_source": f"{peak_kind} HBM copy"},
         "gpu_launches": 2 * K,
-        "gpu_launches": K,
         "timing": "the K timed steps are captured in one CUDA graph (per step: L2 flush read, event, the "
                   "step, event) and replayed once; the two-call figures come from the same protocol, and its "
                   "per-kernel times from a graph with an event between the two kernels",
@@ -442,6 +562,22 @@ def run_ours(args):
         "impl": "ours",
     }
     del r
+    # The step from un-rotated projections: RoPE + append + capture + route in
+    # one launch, then the scan.
+    app = AppendInputs(native, inputs, x)
+    dec_a = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=dev)
+    app_ms, pre_ms = time_append(native, dec_a, x, app, K, args.warmup)
+    if dec_a.workspace.device_error():
+        raise RuntimeError("device error word set by the append-step timing")
+    us_app, _ = aggregate_us(max_over_ranks(sum(app_ms)), K, world)
+    line["append_step"] = {
+        "path": "sr_rope_append_route then sr_decode_attention (RoPE of the query heads and the new key, KV "
+                "append at the last slot, k0/v0 capture, routing and the length update in the first launch)",
+        "us_per_layer_step": round(us_app, 3),
+        "prestep_kernel_us_median": round(statistics.median(pre_ms) * 1e3, 3),
+        "active_units": int(dec_a.active_list[0]),
+        "two_call_us_per_layer_step": round(us_step, 3)}
+    del dec_a
     if world == 1 and not args.no_sweep:
         sweep = []
         for frac in (0.0, 0.25, 0.5, 0.75, 1.0):
@@ -466,6 +602,13 @@ def run_ours(args):
                        "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                        "path": "sr_route_decode_attention, eager launch",
                        "note": "pinned host buffers; every input (caches included) copied each step"}
+        ms_a, h2d_a, d2h_a = e2e_append_measure(native, x, app, max(args.e2e_steps, 50))
+        ms_a = max_over_ranks(ms_a)
+        line["e2e_append"] = {"value": round(ms_a * 1e3 / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d_a,
+                              "d2h_bytes_per_step": d2h_a,
+                              "path": "Decoder.append_step, eager launch, KV cache resident",
+                              "note": "per step: the new token's q/k/v projections host -> device, the output "
+                                      "and route mask device -> host"}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         xc = x.to("cpu")
         us, threads, reps, el = oracle_layer_step_us(xc, args.cpu_budget_s)
