@@ -401,3 +401,43 @@ def test_proxy_quality_analysis_runs_and_matches_oracle_event():
     p0 = proxy_quality.full_attention_p0(x).cpu().view(16, 8, 4).mean(-1)
     near = (p0 - 0.5).abs() < 0.02  # decisions this close to the cutoff may differ by rounding
     assert torch.equal((p0 >= 0.5)[~near], ev_ref[~near])
+
+
+@pytest.mark.parametrize("M,ns,L", [(4, 70, 9000), (8, 40, 6000), (1, 140, 20000), (2, 7, 3000)])
+def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
+    """With forced splits a unit's partials depend only on n_splits and its
+    length, and the last-CTA merge takes them in a fixed order, so unit 0's
+    bits (lse included) must not depend on the rest of the launch: unit 0
+    alone (every CTA holds at most one split, so the merging CTA has no
+    further work) against unit 0 among many active units (more splits than
+    CTAs: CTA j's split j is never its last). ns = 70 at M = 4, 40 at M = 8
+    and 140 at M = 1 take several batches of the merge."""
+    G = native.grid_size()
+    Hkv = 8
+    B = max(1, -(-(G + ns) // (ns * Hkv)) + 1)  # B*Hkv*ns > G + ns
+    x = inputs.make("tiny_4k", seed=7, device=DEV, max_ctx=L)
+    g = torch.Generator(device=DEV).manual_seed(M * 1000 + ns)
+    q = torch.randn((B, Hkv * M, 128), generator=g, device=DEV).to(torch.bfloat16)
+    kc = torch.randn((B, Hkv, L, 128), generator=g, device=DEV).to(torch.bfloat16)
+    vc = torch.randn((B, Hkv, L, 128), generator=g, device=DEV).to(torch.bfloat16)
+    k0, v0 = kc[:, :, 0].contiguous(), vc[:, :, 0].contiguous()
+    sl = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    U = B * Hkv
+    assert U * ns > G + ns and ns <= G
+    del x
+    runs = {}
+    for name, units in (("alone", [0]), ("among_many", list(range(U)))):
+        act = torch.tensor([len(units)] + units, dtype=torch.int32, device=DEV)
+        ws = native.Workspace(B, Hkv * M, Hkv, L, max_splits=ns, device=DEV)
+        lse = torch.empty((B, Hkv * M), dtype=torch.float32, device=DEV)
+        out = native.decode_attention(q, kc, vc, k0, v0, sl, act, n_splits=ns, workspace=ws, lse=lse)
+        torch.cuda.synchronize()
+        assert ws.device_error() == 0
+        runs[name] = (out[0, :M].cpu(), lse[0, :M].cpu())
+    a, b = runs["alone"], runs["among_many"]
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)), "unit 0 depends on the other units"
+    assert torch.equal(a[1].view(torch.int32), b[1].view(torch.int32)), "lse of unit 0 depends on the other units"
+    # and both agree with the oracle
+    ref, _ = oracle.decode(q[:1, :M].cpu(), kc[:1, :1].cpu(), vc[:1, :1].cpu(), v0[:1, :1].cpu(),
+                           sl[:1].cpu(), torch.zeros(1, dtype=torch.uint8))
+    H.assert_active_close(a[0].unsqueeze(0), ref[0].unsqueeze(0), f"M={M} ns={ns}")
