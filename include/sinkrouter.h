@@ -238,6 +238,59 @@ sr_status sr_route_decode_attention(const sr_dims *dims, const void *q, const vo
                                     uint8_t *route_mask, int32_t *active_list, void *out,
                                     void *workspace, size_t workspace_bytes, void *stream);
 
+/* Largest number of parts sr_combine_partials accepts. */
+#define SR_MAX_PARTS 1024
+
+/*
+ * sr_decode_attention_partial -- sr_decode_attention over the positions this
+ * call's cache holds, with each head's result left in the form that combines
+ * across calls over disjoint position ranges (context parallelism: each GPU
+ * holds one contiguous shard of every sequence's cache and scans it; the
+ * shards' results are exchanged and combined with sr_combine_partials). The
+ * README's split-K decode reduces such partials inside one kernel; this is the
+ * same reduction carried across GPUs.
+ *
+ * Arguments are those of sr_decode_attention, with the output replaced by:
+ *   o_part   out fp32 [B, Hq, d]: for an active head, softmax attention over
+ *            the L_b positions of this call's cache, normalised and NOT rounded
+ *            to bf16 (bf16 of it equals sr_decode_attention's out bit for bit);
+ *            for a sink head, v0 widened to fp32 (exact)
+ *   lse_part out fp32 [B, Hq]: natural-log log-sum-exp of the scaled logits
+ *            (q . k_j / sqrt(d)) over those positions; NaN for sink heads
+ * Every rank must route identically (same q, k0, tau) and pass the same active
+ * list; seq_lens holds the lengths of this call's shard (>= 1 each).
+ * Errors: as sr_decode_attention.
+ */
+sr_status sr_decode_attention_partial(const sr_dims *dims, const void *q, const void *k_cache,
+                                      const void *v_cache, const void *k0, const void *v0,
+                                      const int32_t *seq_lens, const int32_t *active_list,
+                                      int32_t n_splits, float *o_part, float *lse_part,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sr_combine_partials -- combine R partial results over disjoint position
+ * ranges into the attention output over their union: per head
+ *     lse = log sum_r exp(lse_r),    out = bf16( sum_r exp(lse_r - lse) o_r )
+ * (the union's softmax denominator is the sum of the parts' denominators). A
+ * head whose part-0 lse is NaN is a sink head and gets bf16(o_0) = v0. A part
+ * with lse = -inf (no positions) weighs 0; if every part does, the output is
+ * undefined.
+ *   dims        batch and n_q_heads give the B*Hq heads (n_kv_heads and
+ *               max_seq_len are not read); head_dim must be 128
+ *   n_parts     R, 1 .. SR_MAX_PARTS
+ *   o_parts     fp32: part r's o_part [B, Hq, d] at o_parts + r * part_stride
+ *   lse_parts   fp32: part r's lse_part [B, Hq] at lse_parts + r * part_stride
+ *   part_stride floats from one part to the next (the same for both arrays): a
+ *               multiple of 4, and >= B*Hq*d when R > 1. A gathered buffer of
+ *               [R][o_part | lse_part] rows uses o_parts = base,
+ *               lse_parts = base + B*Hq*d and its row length as the stride.
+ *   out         bf16 [B, Hq, d]
+ * One launch (one warp per head), asynchronous on `stream`, no workspace.
+ * Errors: SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_CUDA.
+ */
+sr_status sr_combine_partials(const sr_dims *dims, int32_t n_parts, const float *o_parts,
+                              const float *lse_parts, int64_t part_stride, void *out, void *stream);
+
 /* Static description of a status code. */
 const char *sr_status_string(sr_status s);
 

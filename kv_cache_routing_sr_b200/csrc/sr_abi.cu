@@ -1,6 +1,7 @@
 // extern "C" entry points of libsinkrouter.so (declared in include/sinkrouter.h):
 // host-side validation, workspace layout and kernel dispatch. No function here
 // allocates device memory; every buffer is the caller's.
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -203,6 +204,57 @@ sr_status sr_decode_attention_lse(const sr_dims *dims, const void *q, const void
                      dims->max_seq_len, n_splits};
     a.lse = lse;
     const cudaError_t e = sr::launch_decode(a, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+sr_status sr_decode_attention_partial(const sr_dims *dims, const void *q, const void *k_cache, const void *v_cache,
+                                      const void *k0, const void *v0, const int32_t *seq_lens,
+                                      const int32_t *active_list, int32_t n_splits, float *o_part, float *lse_part,
+                                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)k0;
+    const sr_status st = check_dims(dims);
+    if (st != SR_OK)
+        return st;
+    if (!q || !k_cache || !v_cache || !v0 || !seq_lens || !active_list || !o_part || !lse_part)
+        return SR_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(v0, 16) ||
+        !aligned(o_part, 16) || !aligned(seq_lens, 4) || !aligned(active_list, 4) || !aligned(lse_part, 4))
+        return SR_ERR_INVALID_ARG;
+    if (n_splits < 0 || n_splits > SR_MAX_SPLITS)
+        return SR_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256))
+        return SR_ERR_WORKSPACE;
+    const int U = dims->batch * dims->n_kv_heads;
+    const int M = dims->n_q_heads / dims->n_kv_heads;
+    const sr::WorkspaceLayout ws = sr::workspace_layout(U, M, sr::slots_needed(U, n_splits));
+    if (workspace_bytes < ws.total)
+        return SR_ERR_WORKSPACE;
+    sr::DecodeArgs a{q,       k_cache,      v_cache,         v0,         seq_lens,         active_list,
+                     nullptr, workspace,    ws,              dims->batch, dims->n_q_heads, dims->n_kv_heads,
+                     dims->max_seq_len, n_splits};
+    a.lse = lse_part;
+    a.out_f32 = o_part;
+    const cudaError_t e = sr::launch_decode(a, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
+sr_status sr_combine_partials(const sr_dims *dims, int32_t n_parts, const float *o_parts, const float *lse_parts,
+                              int64_t part_stride, void *out, void *stream)
+{
+    // Only the head count and head_dim matter here.
+    if (!dims || dims->batch < 1 || dims->n_q_heads < 1 || (int64_t)dims->batch * dims->n_q_heads > INT32_MAX)
+        return SR_ERR_INVALID_ARG;
+    if (dims->head_dim != sr::kHeadDim)
+        return SR_ERR_UNSUPPORTED;
+    if (!o_parts || !lse_parts || !out || !aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16))
+        return SR_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)dims->batch * dims->n_q_heads;
+    if (n_parts < 1 || n_parts > SR_MAX_PARTS || part_stride % 4 != 0 ||
+        (n_parts > 1 && part_stride < heads * sr::kHeadDim))
+        return SR_ERR_INVALID_ARG;
+    const cudaError_t e = sr::launch_combine((int)heads, n_parts, o_parts, lse_parts, part_stride, out,
+                                             as_stream(stream));
     return e == cudaSuccess ? SR_OK : cuda_fail(e);
 }
 

@@ -109,6 +109,7 @@ struct Params {
     uint8_t *mask_out;   // may be null
     int32_t *active_out; // may be null
     float *lse;          // [B, Hq] natural-log log-sum-exp of the logits; may be null
+    float *out_f32;      // when set, the output is written here in fp32 instead of `out`
 };
 
 template <int RB, int STAGES> struct Cfg {
@@ -555,10 +556,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             if (bitmap[u >> 5] & (1u << (u & 31)))
                 continue;
             const int b = u / p.Hkv, gg = u - b * p.Hkv;
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.v0 + (size_t)u * kHeadDim) + (lane & 15));
-            for (int e = lane; e < M * 16; e += 32) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + (e >> 4)) * kHeadDim);
-                dst[e & 15] = v;
+            const size_t row0 = (size_t)b * p.Hq + (size_t)gg * M;
+            if (p.out_f32) {
+                // fp32 copy of v0 (exact): lane c4 widens elements 4 c4 .. 4 c4 + 3
+                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p.v0 + (size_t)u * kHeadDim) + lane);
+                const float4 f = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                                             __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+                for (int hh = 0; hh < M; ++hh)
+                    reinterpret_cast<float4 *>(p.out_f32 + (row0 + hh) * kHeadDim)[lane] = f;
+            } else {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.v0 + (size_t)u * kHeadDim) + (lane & 15));
+                for (int e = lane; e < M * 16; e += 32) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (row0 + (e >> 4)) * kHeadDim);
+                    dst[e & 15] = v;
+                }
             }
             if (p.lse && lane < M) // no attention was computed for a sink head
                 p.lse[(size_t)b * p.Hq + (size_t)gg * M + lane] = __int_as_float(0x7fc00000);
@@ -589,6 +600,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     int stage = 0;
     uint32_t ph = 0, cph = 0;
     bool ok = true;
+
+    // Final output of one float4 column: acc * inv, in bf16 (round to nearest
+    // even of the same fp32 products) or, for partial outputs, in fp32.
+    auto store_out = [&](int b, int gg, int head, int d4, const float4 &acc, float inv) {
+        const size_t off = ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim + d4;
+        const float4 r = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (p.out_f32) {
+            *reinterpret_cast<float4 *>(p.out_f32 + off) = r;
+        } else {
+            uint2 packed;
+            packed.x = pack_bf16x2(r.x, r.y);
+            packed.y = pack_bf16x2(r.z, r.w);
+            *reinterpret_cast<uint2 *>(p.out + off) = packed;
+        }
+    };
 
     auto cbar_sync = [&]() -> bool {
         __syncwarp();
@@ -859,12 +885,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     if (sgrp == 1) {
                         if (p.lse && d4 == 0)
                             p.lse[(size_t)b * p.Hq + (size_t)gg * M + head] = (m + log2f(l)) * kLn2;
-                        const float inv = 1.f / l;
-                        uint2 packed;
-                        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-                        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-                        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim +
-                                                   d4) = packed;
+                        store_out(b, gg, head, d4, acc, 1.f / l);
                     } else {
                         *reinterpret_cast<float4 *>(comb + 4 * ctid) = acc;
                         *reinterpret_cast<float2 *>(comb + 4 * kMergeThreads + 2 * ctid) = make_float2(m, l);
@@ -892,12 +913,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         }
                         if (p.lse && d4 == 0)
                             p.lse[(size_t)b * p.Hq + (size_t)gg * M + head] = (m + log2f(l)) * kLn2;
-                        const float inv = 1.f / l;
-                        uint2 packed;
-                        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-                        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-                        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + (size_t)gg * M + head) * kHeadDim +
-                                                   d4) = packed;
+                        store_out(b, gg, head, d4, acc, 1.f / l);
                     }
                 }
                 if (ctid == 0)
@@ -1048,6 +1064,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
     p.mask_out = a.mask_out;
     p.active_out = a.active_out;
     p.lse = a.lse;
+    p.out_f32 = a.out_f32;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info->grid);
     cfg.blockDim = dim3(kThreads);

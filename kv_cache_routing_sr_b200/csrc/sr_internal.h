@@ -67,6 +67,9 @@ struct DecodeArgs {
     int32_t *active_out = nullptr;
     // Optional per-head log-sum-exp output (sr_decode_attention_lse).
     float *lse = nullptr;
+    // Partial outputs for context parallelism (sr_decode_attention_partial):
+    // fp32 output instead of `out`.
+    float *out_f32 = nullptr;
 };
 
 // RoPE + append + position-0 capture + routing (sr_rope_append_route).
@@ -84,6 +87,9 @@ struct PrestepArgs {
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);
 cudaError_t launch_rope_append_route(const PrestepArgs &a, cudaStream_t stream);
+// Log-sum-exp combination of n_parts partial outputs (sr_combine_partials).
+cudaError_t launch_combine(int n_heads, int n_parts, const float *o_parts, const float *lse_parts, int64_t part_stride,
+                           void *out, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 // Persistent CTAs of the decode kernel on the current device (0 on error).
 int decode_grid_size();

@@ -41,7 +41,8 @@ _lib = None
 EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_decode_attention",
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
            "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention",
-           "sr_decode_attention_lse", "sr_rope_append_route"]
+           "sr_decode_attention_lse", "sr_rope_append_route", "sr_decode_attention_partial",
+           "sr_combine_partials"]
 
 
 def load(path: str = LIBRARY):
@@ -83,6 +84,10 @@ def load(path: str = LIBRARY):
     lib.sr_rope_append_route.argtypes = [dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                          vp, vp, vp]
     lib.sr_rope_append_route.restype = ctypes.c_int
+    lib.sr_decode_attention_partial.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, u64, vp]
+    lib.sr_decode_attention_partial.restype = ctypes.c_int
+    lib.sr_combine_partials.argtypes = [dp, i32, vp, vp, ctypes.c_int64, vp, vp]
+    lib.sr_combine_partials.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -183,6 +188,48 @@ def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=Non
     else:
         _check("sr_decode_attention_lse",
                load().sr_decode_attention_lse(*common, _dev(lse, "lse", torch.float32), *tail))
+    return out
+
+
+def decode_attention_partial(q, k_cache, v_cache, k0, v0, seq_lens, active_list, o_part=None, lse_part=None,
+                             n_splits: int = 0, workspace: Workspace | None = None, stream=None):
+    """sr_decode_attention_partial: the scan over this cache's positions with
+    fp32 normalised outputs o_part [B, Hq, 128] and natural-log lse_part [B, Hq]
+    (NaN for sink heads), ready for combine_partials. Returns (o_part, lse_part)."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if o_part is None:
+        o_part = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = Workspace(B, Hq, Hkv, Lmax, n_splits, device=q.device)
+    dims = dims_of(B, Hq, Hkv, Lmax, d)
+    k0p = _dev(k0, "k0", torch.bfloat16) if k0 is not None else None
+    st = load().sr_decode_attention_partial(
+        ctypes.byref(dims), _dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+        _dev(v_cache, "v_cache", torch.bfloat16), k0p, _dev(v0, "v0", torch.bfloat16),
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(active_list, "active_list", torch.int32), int(n_splits),
+        _dev(o_part, "o_part", torch.float32), _dev(lse_part, "lse_part", torch.float32),
+        ctypes.c_void_p(workspace.ptr), workspace.nbytes, _stream(stream))
+    _check("sr_decode_attention_partial", st)
+    return o_part, lse_part
+
+
+def combine_partials(o_parts, lse_parts, part_stride: int, n_parts: int, batch: int, n_q_heads: int, out=None,
+                     stream=None):
+    """sr_combine_partials over n_parts parts laid out part_stride floats apart:
+    o_parts / lse_parts are fp32 CUDA tensors whose storage starts at part 0's
+    o_part / lse_part. Returns out bf16 [B, Hq, 128]."""
+    if out is None:
+        out = torch.empty((batch, n_q_heads, HEAD_DIM), dtype=torch.bfloat16, device=o_parts.device)
+    for t, name in ((o_parts, "o_parts"), (lse_parts, "lse_parts")):
+        if not t.is_cuda or t.dtype != torch.float32:
+            raise ValueError(f"{name} must be a float32 CUDA tensor")
+    dims = dims_of(batch, n_q_heads, n_q_heads, 1)  # only B, Hq and head_dim are read
+    st = load().sr_combine_partials(ctypes.byref(dims), int(n_parts), o_parts.data_ptr(), lse_parts.data_ptr(),
+                                    int(part_stride), _dev(out, "out", torch.bfloat16), _stream(stream))
+    _check("sr_combine_partials", st)
     return out
 
 
