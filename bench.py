@@ -212,7 +212,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # our arm
 
-def _captured_steps(native, dec, x, tau, steps, flush, split_events, fused):
+def _captured_steps(native, dec, x, tau, steps, flush, split_events, fused, rotate=None):
     """Capture `steps` layer-steps in ONE CUDA graph, as a decode forward would
     run them: before each step an L2 flush (a 256 MiB read), then an event and
     the step, then an event. The step is either the single fused launch
@@ -223,25 +223,30 @@ def _captured_steps(native, dec, x, tau, steps, flush, split_events, fused):
     import torch
     # external events: recorded as timestamps by the graph's event nodes
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
-    args = (x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens)
+    xs = rotate or [x]
     side = torch.cuda.Stream(device=x.q.device)
     side.wait_stream(torch.cuda.current_stream(x.q.device))
     with torch.cuda.stream(side):  # warm-up outside the capture
-        dec.step(*args, tau)
-        dec.step_fused(*args, tau)
-        flush.sum()
+        for xi in xs:
+            dec.step(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, tau)
+            dec.step_fused(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, tau)
+        if flush is not None:
+            flush.sum()
     torch.cuda.current_stream(x.q.device).wait_stream(side)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         st = torch.cuda.current_stream()
         for i in range(steps):
-            flush.sum()
+            xi = xs[i % len(xs)]
+            args = (xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens)
+            if flush is not None:
+                flush.sum()
             ev[i][0].record(st)
             if fused:
                 native.route_decode_attention(*args, tau, dec.out, dec.route_mask, dec.active_list, 0,
                                               dec.workspace)
             else:
-                native.route(x.q, x.k0, tau, dec.route_mask, dec.active_list)
+                native.route(xi.q, xi.k0, tau, dec.route_mask, dec.active_list)
                 if split_events:
                     ev[i][1].record(st)
                 native.decode_attention(*args, dec.active_list, dec.out, 0, dec.workspace)
@@ -249,11 +254,12 @@ def _captured_steps(native, dec, x, tau, steps, flush, split_events, fused):
     return g, ev
 
 
-def time_steps(native, dec, x, tau, steps, warmup, flush, barrier, fused):
-    """Per-step device times (ms): events bracket the step only."""
+def time_steps(native, dec, x, tau, steps, warmup, flush, barrier, fused, rotate=None):
+    """Per-step device times (ms): events bracket the step only. flush=None
+    skips the L2 flush; `rotate` cycles the steps over several input sets."""
     import torch
-    gw, _ = _captured_steps(native, dec, x, tau, warmup, flush, False, fused)
-    g, ev = _captured_steps(native, dec, x, tau, steps, flush, False, fused)
+    gw, _ = _captured_steps(native, dec, x, tau, warmup, flush, False, fused, rotate)
+    g, ev = _captured_steps(native, dec, x, tau, steps, flush, False, fused, rotate)
     gw.replay()
     barrier()
     torch.cuda.synchronize()
@@ -354,6 +360,47 @@ def time_append(native, dec, x, a, steps, warmup):
     pre_ms = [e[0].elapsed_time(e[1]) for e in evk]
     del flush
     return steps_ms, pre_ms
+
+
+def measure_config(native, inputs, name, steps, warmup, flush, device, peak, l2_mode="flush", copies=1):
+    """Routed and routing-disabled two-call steps of one more workload, for the
+    other_configs block. l2_mode: "flush" (a 256 MiB read before every step),
+    "hot" (no flush, the same inputs every step) or "rotate" (no flush; the
+    steps cycle over `copies` independently seeded input sets whose caches
+    together exceed L2)."""
+    import torch
+    xs = [inputs.make(name, seed=100 + c, device=device) for c in range(copies if l2_mode == "rotate" else 1)]
+    x = xs[0]
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=device)
+    fl = flush if l2_mode == "flush" else None
+    rot = xs if l2_mode == "rotate" else None
+    nobar = lambda: None  # noqa: E731
+    routed = time_steps(native, dec, x, x.tau, steps, warmup, fl, nobar, False, rot)
+    disabled = time_steps(native, dec, x, float("inf"), steps, warmup, fl, nobar, False, rot)
+    if dec.workspace.device_error():
+        raise RuntimeError(f"device error word set on {name}")
+    needs, needs_all, acts = [], [], []
+    for xi in xs:
+        dec.step(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, xi.tau)
+        act = active_units_of(dec.active_list.cpu())
+        sl = xi.seq_lens.cpu().tolist()
+        needs.append(inputs.needed_bytes(sl, act, xi.n_kv_heads, xi.n_q_heads, xi.batch))
+        needs_all.append(inputs.needed_bytes(sl, range(xi.batch * xi.n_kv_heads), xi.n_kv_heads, xi.n_q_heads,
+                                             xi.batch))
+        acts.append(len(act))
+    need, need_all = statistics.mean(needs), statistics.mean(needs_all)
+    us, us_dis = statistics.mean(routed) * 1e3, statistics.mean(disabled) * 1e3
+    gbs = need / (us * 1e-6) / 1e9
+    gbs_dis = need_all / (us_dis * 1e-6) / 1e9
+    out = {"workload": name, "l2": l2_mode + (f" over {copies} input sets" if l2_mode == "rotate" else ""),
+           "us_per_layer_step": round(us, 3), "us_p50": round(statistics.median(routed) * 1e3, 3),
+           "needed_bytes": int(need), "effective_gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peak, 4),
+           "active_units": acts[0] if len(set(acts)) == 1 else acts, "units": x.batch * x.n_kv_heads,
+           "routing_disabled_us": round(us_dis, 3), "routing_disabled_gbs": round(gbs_dis, 1),
+           "speedup_routed": round(us_dis / us, 3)}
+    del xs, x, dec
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_workload(native, inputs, x, steps, warmup, flush, barrier, fused=True):
@@ -458,15 +505,18 @@ def e2e_append_measure(native, x, a, steps):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def oracle_layer_step_us(x_cpu, budget_s, min_reps=1):
-    """The fp64 oracle, as it stands, on whole layer-steps of this workload."""
+def oracle_layer_step_us(x_cpu, budget_s, min_reps=1, threads=None):
+    """The fp64 oracle, as it stands, on whole layer-steps of this workload,
+    with `threads` threads (default: one per active unit, capped at the host
+    cores; the oracle splits whole units over its threads)."""
     import torch
 
     import oracle
     tau = float(torch.tensor(x_cpu.tau, dtype=torch.float32))
     mask, active, _ = oracle.route(x_cpu.q, x_cpu.k0, tau)
     n_act = int(active[0])
-    threads = max(1, min(os.cpu_count() or 1, max(1, n_act)))
+    if threads is None:
+        threads = max(1, min(os.cpu_count() or 1, max(1, n_act)))
     reps = 0
     t0 = time.perf_counter()
     while True:
@@ -595,6 +645,17 @@ def run_ours(args):
             del x5, s5
             torch.cuda.empty_cache()
         line["sweep_512k"] = sweep
+    if world == 1 and not args.no_sweep:
+        # The remaining workloads: tiny 4K with L2 hot and cold (rotating over
+        # input sets that together exceed L2), the ragged 70B-shaped and the
+        # LLaVA-shaped layers with the flush protocol.
+        oc_steps = max(20, min(K, 50))
+        line["other_configs"] = [
+            measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "hot"),
+            measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "rotate", copies=12),
+            measure_config(native, inputs, "llama70b_ragged", oc_steps, args.warmup, flush, dev, peak),
+            measure_config(native, inputs, "llava7b_mha", oc_steps, args.warmup, flush, dev, peak),
+        ]
     if not args.no_e2e:
         ms, h2d, d2h = e2e_measure(native, x, args.e2e_steps)
         ms = max_over_ranks(ms)
@@ -612,11 +673,14 @@ def run_ours(args):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         xc = x.to("cpu")
         us, threads, reps, el = oracle_layer_step_us(xc, args.cpu_budget_s)
+        us1, _, reps1, el1 = oracle_layer_step_us(xc, args.cpu_budget_s / 2, threads=1)
         line["cpu_baseline"] = {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"{reps} whole layer-steps of {x.workload.name} "
                                           f"({x.batch * x.n_kv_heads} units) in {el:.1f} s, fp64 C oracle, "
                                           f"{threads} threads (one per active unit, capped at the host cores)",
-                                "host_cores": os.cpu_count()}
+                                "host_cores": os.cpu_count(),
+                                "one_thread": {"value": round(us1, 1), "unit": UNIT,
+                                               "sample": f"{reps1} layer-steps in {el1:.1f} s"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
