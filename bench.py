@@ -59,6 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-sweep", action="store_true", help="skip the 512K sink-fraction sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--context-parallel", action="store_true",
+                    help="instead of the contract line: one 512K layer-step (half the groups sinks) sharded over "
+                         "the --gpus ranks by position: partial scans, one all-gather, the combine (strong scaling)")
     ap.add_argument("--multilayer", action="store_true",
                     help="instead of the contract line: per-token attention latency of a 32-layer stack, "
                          "CUDA-graph captured, at 128K/256K/512K context, routed vs routing disabled")
@@ -805,8 +808,96 @@ def run_proxy_quality(args):
     print(json.dumps(out), flush=True)
 
 
+def run_context_parallel(args):
+    """Context-parallel layer-step: every rank scans its shard of the 512K
+    sequence, the ranks all-gather their (o, lse) rows and every rank combines
+    them. Per step: L2 flush, event, route + partial scan, event, all-gather +
+    combine, event; eager launches (the collective stays out of CUDA graphs).
+    Time is the max over ranks."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from kv_cache_routing_sr_b200 import context_parallel as cp
+    from kv_cache_routing_sr_b200 import inputs
+
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peak, peak_kind = hbm_peak()
+    x = inputs.make("llama8b_512k", seed=args.seed, device=dev, sink_fraction=0.5)
+    bounds = cp.shard_bounds(x.seq_lens.tolist(), world)
+    ks, vs = cp.shard_cache(x.k_cache, bounds[rank]), cp.shard_cache(x.v_cache, bounds[rank])
+    lens = torch.tensor([e - s for s, e in bounds[rank]], dtype=torch.int32, device=dev)
+    q, k0, v0, tau = x.q, x.k0, x.v0, x.tau
+    need = None
+    d = cp.ContextParallelDecoder(x.batch, x.n_q_heads, x.n_kv_heads, ks.shape[2], world=world, device=dev)
+    d.step(q, ks, vs, k0, v0, lens, tau)
+    torch.cuda.synchronize()
+    act = active_units_of(d.dec.active_list.cpu())
+    need = inputs.needed_bytes(x.seq_lens.tolist(), act, x.n_kv_heads, x.n_q_heads, x.batch)
+    del x
+    torch.cuda.empty_cache()
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        d.step(q, ks, vs, k0, v0, lens, tau)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    st = torch.cuda.current_stream()
+    for i in range(K):
+        flush.sum()
+        ev[i][0].record(st)
+        d.local(q, ks, vs, k0, v0, lens, tau)
+        ev[i][1].record(st)
+        d.finish()
+        ev[i][2].record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    tot = [e[0].elapsed_time(e[2]) for e in ev]
+    loc = [e[0].elapsed_time(e[1]) for e in ev]
+    fin = [e[1].elapsed_time(e[2]) for e in ev]
+    err = d.dec.workspace.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err}")
+    us = reduce_max(sum(tot), dev, world) / K * 1e3
+    us_loc = reduce_max(sum(loc), dev, world) / K * 1e3
+    us_fin = reduce_max(sum(fin), dev, world) / K * 1e3
+    if rank == 0:
+        gbs = need / (us * 1e-6) / 1e9
+        line = {"metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": round(us / 1e3, 6), "higher_is_better": False,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
+                "config": {"workload": "llama8b_512k", "sink_fraction": 0.5, "batch": 1, "context": 524288,
+                           "q_heads": 32, "kv_heads": 8, "head_dim": 128, "tau": 0.6, "active_units": len(act),
+                           "parallelism": f"cp{world} (positions sharded; one all-gather of (o, lse) per step)",
+                           "l2": "256 MiB read before every step"},
+                "mode": "context_parallel", "impl": "ours",
+                "effective_gbs": round(gbs, 1), "frac_of_hbm_peak_whole_job": round(gbs / (peak * world), 4),
+                "local_us": round(us_loc, 3), "exchange_and_combine_us": round(us_fin, 3),
+                "row_bytes_per_rank": d.stride * 4, "timing": "eager launches, CUDA events per step, max over ranks",
+                "peak_source": f"{peak_kind} HBM copy"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.context_parallel:
+        if args.impl == "reference":
+            raise SystemExit("--context-parallel has no reference arm")
+        run_context_parallel(args)
+        return
     if args.proxy_quality:
         run_proxy_quality(args)
         return
