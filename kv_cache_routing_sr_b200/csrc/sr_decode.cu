@@ -66,6 +66,7 @@ constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeThreads = 32 * kCWarps;
+constexpr int kCosBuf = kCWarps * kMaxGroup * kHeadDim; // floats of the comb scratch, reused by fused routing
 constexpr int kMergeBatch = 16; // partials in flight per thread in the final merge
 
 struct alignas(16) TileHdr {
@@ -124,12 +125,15 @@ template <int RB, int STAGES> struct Cfg {
     static constexpr int OFF_BAR = OFF_HDR + STAGES * (int)sizeof(TileHdr);
     static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
     static constexpr int OFF_BITMAP = OFF_MISC + 256;
-    static constexpr int BYTES = OFF_BITMAP + SR_MAX_UNITS / 8;
+    // seq_lens staged outside the stage buffers: the producer reads it while
+    // the copies run
+    static constexpr int OFF_SEQ = OFF_BITMAP + SR_MAX_UNITS / 8;
+    static constexpr int BYTES = OFF_SEQ + kSeqTab * 4;
     static constexpr int ALLOC = BYTES + 1024; // room to align the base to 1024 B
     static_assert(sizeof(Misc) <= 256, "misc block");
-    // Prologue tables (seq_lens, active lengths, active units) live in the
+    // Prologue tables (active lengths, active units, sink flags) live in the
     // stage buffers before the first copy is issued.
-    static_assert(kSeqTab * 4 + SR_MAX_UNITS * 7 <= STAGES * STAGE, "prologue tables");
+    static_assert(SR_MAX_UNITS * 7 <= STAGES * STAGE, "prologue tables");
     static_assert(BN <= 256, "TMA box rows");
     static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
 };
@@ -152,10 +156,11 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 // Sequence length of unit u, clamped to [1, Lmax] (the prologue reports the
-// clamp; every later lookup must give the same value).
-__device__ __forceinline__ int unit_len(const Params &p, int u)
+// clamp; every later lookup must give the same value), from the shared table
+// when the batch fits it.
+__device__ __forceinline__ int unit_len(const Params &p, int u, const int32_t *seqtab)
 {
-    const int L = __ldg(p.seq_lens + u / p.Hkv);
+    const int L = seqtab ? seqtab[u / p.Hkv] : __ldg(p.seq_lens + u / p.Hkv);
     return L < 1 ? 1 : (L > p.Lmax ? p.Lmax : L);
 }
 
@@ -202,30 +207,54 @@ __device__ __forceinline__ long long block_scan(long long x, Misc *misc, long lo
     return before + v;
 }
 
-// Fused routing, one pass per kThreads (unit, head) pairs: sflag[u] = sink.
-// Every CTA computes the same decisions as the routing kernel (same
-// arithmetic, sr_route_math.cuh); CTA 0 also writes the route mask.
+// Fused routing: sflag[u] = sink for every unit, read straight from global
+// memory, one half-warp per (unit, head) pair. Every CTA computes the same
+// decisions as the routing kernel (the same arithmetic, sr_route_math.cuh);
+// CTA 0 also writes the route mask.
 template <int M>
-__device__ __forceinline__ void route_units(const Params &p, int U, uint8_t *sflag)
+__device__ __forceinline__ void route_units(const Params &p, int U, uint8_t *sflag, float *cosbuf)
 {
-    const int pairs = U * M;
-    for (int base = 0; base < pairs; base += kThreads) {
-        const int pr = base + (int)threadIdx.x;
-        const bool valid = pr < pairs;
-        const int u = pr / M, m = pr - (pr / M) * M;
-        float c = INFINITY;
-        if (valid) {
-            const int b = u / p.Hkv, g = u - b * p.Hkv;
-            c = head_cosine(p.q + ((size_t)b * p.Hq + (size_t)g * M + m) * kHeadDim, p.k0 + (size_t)u * kHeadDim,
-                            pr & 15);
+    // Units in chunks whose cosines fit cosbuf (kCosBuf floats); per round each
+    // half-warp loads the blocks of 4 pairs before reducing any of them.
+    constexpr int kChunkUnits = kCosBuf / M;
+    constexpr int kHalfWarps = kThreads / 16;
+    const int hw = (int)threadIdx.x >> 4, l16 = (int)threadIdx.x & 15;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int u0 = 0; u0 < U; u0 += kChunkUnits) {
+        const int nu = (U - u0) < kChunkUnits ? (U - u0) : kChunkUnits;
+        const int pairs = nu * M;
+        for (int base = 0; base < pairs; base += 4 * kHalfWarps) {
+            uint4 qv[4], kv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int pr = base + r * kHalfWarps + hw;
+                const bool valid = pr < pairs;
+                // q row (u0*M + pr) of [B*Hq, 128]; k0 row of unit u0 + pr/M
+                qv[r] = valid ? __ldg(reinterpret_cast<const uint4 *>(p.q + ((size_t)u0 * M + pr) * kHeadDim) + l16)
+                              : zero;
+                kv[r] = valid ? __ldg(reinterpret_cast<const uint4 *>(p.k0 + ((size_t)u0 + pr / M) * kHeadDim) + l16)
+                              : zero;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int pr = base + r * kHalfWarps + hw;
+                const float c = pair_cosine(qv[r], kv[r]);
+                if (pr < pairs && l16 == 0)
+                    cosbuf[pr] = c;
+            }
         }
-        c = group_min<M>(c);
-        if (valid && m == 0) {
-            const uint8_t sink = (c >= p.tau) ? 1 : 0;
-            sflag[u] = sink;
+        __syncthreads();
+        for (int lu = (int)threadIdx.x; lu < nu; lu += kThreads) {
+            float s = INFINITY;
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                s = fminf(s, cosbuf[lu * M + m]);
+            const uint8_t sink = (s >= p.tau) ? 1 : 0;
+            sflag[u0 + lu] = sink;
             if (blockIdx.x == 0 && p.mask_out)
-                p.mask_out[u] = sink;
+                p.mask_out[u0 + lu] = sink;
         }
+        __syncthreads();
     }
 }
 
@@ -276,11 +305,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     // Prologue tables in the stage buffers (free until the first copy),
     // sized by the actual batch and unit count.
     const bool seq_smem = p.B <= kSeqTab;
-    const int seq_bytes = seq_smem ? ((4 * p.B + 127) & ~127) : 0;
-    int32_t *seqtab = reinterpret_cast<int32_t *>(smem);
-    int32_t *ltab = reinterpret_cast<int32_t *>(smem + seq_bytes);
-    int16_t *utab = reinterpret_cast<int16_t *>(smem + seq_bytes + ((4 * U + 127) & ~127));
-    uint8_t *sflag = smem + seq_bytes + ((4 * U + 127) & ~127) + ((2 * U + 127) & ~127);
+    int32_t *seqtab = reinterpret_cast<int32_t *>(smem + C::OFF_SEQ);
+    int32_t *ltab = reinterpret_cast<int32_t *>(smem);
+    int16_t *utab = reinterpret_cast<int16_t *>(smem + ((4 * U + 127) & ~127));
+    uint8_t *sflag = smem + ((4 * U + 127) & ~127) + ((2 * U + 127) & ~127);
     int errbits = 0;
     int n = 0;
     long long local = 0;
@@ -342,16 +370,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         // measured slower: 148 CTAs copying the same few KB serialise.)
         switch (M) {
         case 1:
-            route_units<1>(p, U, sflag);
+            route_units<1>(p, U, sflag, comb);
             break;
         case 2:
-            route_units<2>(p, U, sflag);
+            route_units<2>(p, U, sflag, comb);
             break;
         case 4:
-            route_units<4>(p, U, sflag);
+            route_units<4>(p, U, sflag, comb);
             break;
         default:
-            route_units<8>(p, U, sflag);
+            route_units<8>(p, U, sflag, comb);
             break;
         }
         __syncthreads();
@@ -505,7 +533,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     const int u = unit_at(i);
                     if (u < 0 || u >= U)
                         break;
-                    const int L = unit_len(p, u);
+                    const int L = unit_len(p, u, seq_smem ? seqtab : nullptr);
                     const long long b0 = (r0 > S ? r0 : S) - S;
                     const long long e0 = (r1 < S + L ? r1 : S + L) - S;
                     const long long cf = S / chunk, cl = (S + L - 1) / chunk;
@@ -521,7 +549,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 const int u = unit_at(i);
                 if (u < 0 || u >= U)
                     break;
-                const int L = unit_len(p, u);
+                const int L = unit_len(p, u, seq_smem ? seqtab : nullptr);
                 const long long b0 = (long long)s * L / ns, e0 = (long long)(s + 1) * L / ns;
                 ok = emit_split(u, b0, e0, (int)j, ns, i * ns);
             }
@@ -815,16 +843,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 }
                 __stcg(p.part_ml + (size_t)h.slot * M + ctid, make_float2(Mh, Lh));
             }
-            __threadfence();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
             mrun[0] = mrun[1] = -INFINITY;
             lrun[0] = lrun[1] = 0.f;
+            // Publish the partial: the consumer barrier orders every thread's
+            // stores before thread 0's gpu-scope release, which the last
+            // arriving CTA's acquire (the same atomic) pairs with; its own
+            // barrier then orders the acquire before every thread's merge
+            // loads. No separate fences.
             if (!(ok = cbar_sync()))
                 break;
             if (ctid == 0)
-                misc->is_last = (atomicAdd(p.cnt + h.unit, 1) == h.nseg - 1) ? 1 : 0;
+                misc->is_last = (atom_add_acq_rel_gpu(p.cnt + h.unit, 1) == h.nseg - 1) ? 1 : 0;
             if (!(ok = cbar_sync()))
                 break;
             if (misc->is_last) {
@@ -834,7 +866,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 // Each thread keeps kMergeBatch partials in flight; the merge
                 // order is fixed, so the result does not depend on which CTA
                 // finished last.
-                __threadfence();
                 const int b = h.unit / p.Hkv, gg = h.unit - b * p.Hkv;
                 const int ncol = M * 32;
                 const int cpg = ncol < kMergeThreads ? ncol : kMergeThreads;

@@ -26,9 +26,9 @@
 // key rotate it (each takes 8 elements and their 8 partners), write the cache
 // slot, and stage the group's position-0 key (the captured one at slot 0, else
 // the stored k0); eight threads per query row rotate it into q_out and the
-// staged rows; the staged rows are routed with the same routine and the same
-// per-pair visiting order as the routing kernel, so the decision equals
-// sr_route on (q_out, k0) bit for bit. Lengths advance after every read of
+// staged rows; the staged rows are routed with the routing kernel's own
+// routine (one half-warp per pair), so the decision equals sr_route on
+// (q_out, k0) bit for bit. Lengths advance after every read of
 // them; the compaction is the routing kernel's.
 #include <atomic>
 #include <cuda_bf16.h>
@@ -46,7 +46,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 160 * 1024; // shared bytes for staged q / k0 rows
 
-template <int M> constexpr int chunk_units() { return kRowBudget / ((M + 1) * 256); }
+template <int M> __host__ __device__ constexpr int chunk_units() { return kRowBudget / ((M + 1) * 256); }
 
 struct PrestepParams {
     const __nv_bfloat16 *q_in, *k_new, *v_new;
@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
     extern __shared__ __align__(128) uint8_t dsm[]; // [cu*(M+1)*256 staged rows][B*Hkv sink flags]
     __shared__ int32_t warp_cnt[kWarps];
     __shared__ int32_t warp_off[kWarps + 1];
+    __shared__ float cosbuf[chunk_units<M>() * M];
 
     const int U = p.B * p.Hkv;
     uint4 *rows = reinterpret_cast<uint4 *>(dsm);
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
             qd[j + 8] = hi;
         }
         __syncthreads();
-        route_staged<M, kThreads>(rows, u0, nu, p.tau, sink_flag, p.mask);
+        route_staged<M, kThreads>(rows, u0, nu, p.tau, sink_flag, p.mask, cosbuf);
         __syncthreads(); // the rows are overwritten by the next chunk
     }
 

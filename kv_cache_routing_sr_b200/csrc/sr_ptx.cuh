@@ -114,6 +114,14 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// atomicAdd with acquire-release semantics at gpu scope; returns the old value.
+__device__ __forceinline__ int32_t atom_add_acq_rel_gpu(int32_t *addr, int32_t v)
+{
+    int32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+    return old;
+}
+
 // ---- warp-level matrix fragments ---------------------------------------------------------
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr)

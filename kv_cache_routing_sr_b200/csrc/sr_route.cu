@@ -10,8 +10,9 @@
 //
 // Layout: one CTA of 256 threads. The q and k0 rows of a chunk of units (all
 // units, for every workload here) are staged in shared memory by two bulk
-// copies, then one thread per (unit, query head) pair computes the cosine and
-// the group minimum is a shuffle over adjacent lanes. The compaction writes
+// copies, then one half-warp per (unit, query head) pair computes the cosine
+// (16 lanes of 8 elements each and a shuffle tree) and one thread per unit
+// takes the minimum over its heads. The compaction writes
 // active units in ascending order with warp ballots and a block prefix, so no
 // CTA of the decode kernel is ever bound to a sink unit.
 #include <atomic>
@@ -33,13 +34,13 @@ constexpr int kRowBudget = 160 * 1024; // shared bytes for staged q / k0 rows
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Units per staged chunk for group size M.
-template <int M> constexpr int chunk_units() { return kRowBudget / ((M + 1) * 256); }
+template <int M> __host__ __device__ constexpr int chunk_units() { return kRowBudget / ((M + 1) * 256); }
 
 // M = query heads per KV head (compile time). The q rows of a chunk of units
 // and their k0 rows are contiguous in global memory, so one thread stages them
 // with two bulk copies (one memory round trip, whatever the chunk size); then
-// one thread per (unit, head) pair computes the cosine from shared memory and
-// the M lanes of a unit take the minimum with shuffles.
+// each half-warp computes one (unit, head) cosine from shared memory and one
+// thread per unit takes the minimum over its heads.
 template <int M>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k0, float tau,
@@ -49,6 +50,7 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
     __shared__ __align__(8) uint64_t bar;
     __shared__ int32_t warp_cnt[kRouteWarps];
     __shared__ int32_t warp_off[kRouteWarps + 1];
+    __shared__ float cosbuf[chunk_units<M>() * M];
 
     const int U = B * Hkv;
     uint4 *rows = reinterpret_cast<uint4 *>(dsm);
@@ -89,7 +91,7 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
             timed_out = true;
             break;
         }
-        route_staged<M, kRouteThreads>(rows, u0, nu, tau, sink_flag, mask);
+        route_staged<M, kRouteThreads>(rows, u0, nu, tau, sink_flag, mask, cosbuf);
         __syncthreads(); // the rows are overwritten by the next chunk
     }
     if (timed_out) {

@@ -9,123 +9,92 @@
 
 namespace sr {
 
-// <a,b>, <a,a> and <b,b> of two rows of 128 bf16 held as 16 x 16-byte vectors,
-// in one pass (each vector is used once, so all 32 loads can be in flight).
-__device__ __forceinline__ void dots_row(const uint4 (&a)[16], const uint4 (&b)[16], float &ab, float &aa, float &bb)
+// The cosine of a (unit, head) pair is computed by the 16 lanes of a
+// half-warp: lane l takes the 16-byte block l (elements 8l .. 8l+7) of the
+// query row and of the key row, sums its 8 products in element order, and a
+// fixed xor-shuffle tree (offsets 8, 4, 2, 1) adds the 16 lane sums. Every
+// caller uses this one arithmetic, so they all take the same decision bit for
+// bit.
+
+// Lane sums of <a,b>, <a,a> and <b,b> over one 16-byte block (8 bf16) of each row.
+__device__ __forceinline__ void dots_vec(const uint4 &a, const uint4 &b, float &ab, float &aa, float &bb)
 {
     ab = aa = bb = 0.f;
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const uint32_t aw[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
-        const uint32_t bw[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[j]));
-            const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bw[j]));
-            ab = fmaf(fa.x, fb.x, ab);
-            ab = fmaf(fa.y, fb.y, ab);
-            aa = fmaf(fa.x, fa.x, aa);
-            aa = fmaf(fa.y, fa.y, aa);
-            bb = fmaf(fb.x, fb.x, bb);
-            bb = fmaf(fb.y, fb.y, bb);
-        }
+    for (int j = 0; j < 4; ++j) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[j]));
+        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bw[j]));
+        ab = fmaf(fa.x, fb.x, ab);
+        ab = fmaf(fa.y, fb.y, ab);
+        aa = fmaf(fa.x, fa.x, aa);
+        aa = fmaf(fa.y, fa.y, aa);
+        bb = fmaf(fb.x, fb.x, bb);
+        bb = fmaf(fb.y, fb.y, bb);
     }
 }
 
-// cos(q_h, k0_g) in fp32 for query row `qrow` and key row `krow` (128 bf16
-// each), read straight from global memory; 0 when a norm is 0; a NaN result is
-// returned as +inf so that it never lowers the group minimum. The 16 vectors
-// of a row are combined in the same rotated order as head_cosine_smem, so both
-// give the same bits for the same `rot`.
-__device__ __forceinline__ float head_cosine(const __nv_bfloat16 *__restrict__ qrow,
-                                             const __nv_bfloat16 *__restrict__ krow, int rot)
+// Sum over the 16 lanes of each half-warp; every lane receives it. All 32
+// lanes of the warp must call it.
+__device__ __forceinline__ float half_warp_sum(float x)
 {
-    uint4 qa[16], ka[16];
-    const uint4 *qv = reinterpret_cast<const uint4 *>(qrow);
-    const uint4 *kv = reinterpret_cast<const uint4 *>(krow);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        qa[i] = __ldg(qv + ((i + rot) & 15));
-        ka[i] = __ldg(kv + ((i + rot) & 15));
-    }
-    float dot, qq, kk;
-    dots_row(qa, ka, dot, qq, kk);
-    float c = (qq == 0.f || kk == 0.f) ? 0.f : dot / (sqrtf(qq) * sqrtf(kk));
-    if (c != c)
-        c = INFINITY;
-    return c;
+    for (int off = 8; off > 0; off >>= 1)
+        x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
 }
 
-// cos(q_h, k0_g) from rows staged in shared memory (128 bf16 = 16 x 16-byte
-// vectors each). The vectors are visited starting at `rot` (mod 16), taken from
-// the pair index so that adjacent threads hit different shared-memory banks;
-// the visiting order fixes the fp32 rounding, so every caller that uses the
-// same pair index gets the same bits. Same conventions as head_cosine.
-__device__ __forceinline__ float head_cosine_smem(const uint4 *qrow, const uint4 *krow, int rot)
+// cos(q_h, k0_g) of one pair from this lane's blocks: 0 when a norm is 0; a
+// NaN result is returned as +inf so that it never lowers the group minimum.
+// Returned in all 16 lanes of the half-warp. All 32 lanes must call it.
+__device__ __forceinline__ float pair_cosine(const uint4 &qv, const uint4 &kv)
 {
-    float ab = 0.f, aa = 0.f, bb = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int k = (i + rot) & 15;
-        const uint4 av = qrow[k], bv = krow[k];
-        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[j]));
-            const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bw[j]));
-            ab = fmaf(fa.x, fb.x, ab);
-            ab = fmaf(fa.y, fb.y, ab);
-            aa = fmaf(fa.x, fa.x, aa);
-            aa = fmaf(fa.y, fa.y, aa);
-            bb = fmaf(fb.x, fb.x, bb);
-            bb = fmaf(fb.y, fb.y, bb);
-        }
-    }
+    float ab, aa, bb;
+    dots_vec(qv, kv, ab, aa, bb);
+    ab = half_warp_sum(ab);
+    aa = half_warp_sum(aa);
+    bb = half_warp_sum(bb);
     float c = (aa == 0.f || bb == 0.f) ? 0.f : ab / (sqrtf(aa) * sqrtf(bb));
     if (c != c)
         c = INFINITY;
     return c;
 }
 
-// Minimum over groups of M adjacent lanes (M divides 32).
-template <int M> __device__ __forceinline__ float group_min(float c)
-{
-#pragma unroll
-    for (int off = 1; off < M; off <<= 1)
-        c = fminf(c, __shfl_xor_sync(0xffffffffu, c, off));
-    return c;
-}
-
-} // namespace sr
-
-namespace sr {
-
 // Route the nu units u0 .. u0+nu-1 whose rows are staged in shared memory:
 // `rows` holds their nu*M query rows (row u*M+m of q) followed by their nu key
-// rows, 256 bytes each. NT threads take one (unit, head) pair each per pass
-// (NT a multiple of 32, so a unit's M pairs sit in adjacent lanes of one
-// warp). Writes sflag[u] = sink, and mask_out[u] when mask_out is not null.
+// rows, 256 bytes each. NT threads (a multiple of 32) take NT/16 pairs per
+// pass, one per half-warp; the pairs' cosines go to cosbuf (nu*M floats), and
+// after a block barrier one thread per unit takes the minimum over its M heads.
+// Writes sflag[u] = sink, and mask_out[u] when mask_out is not null. Called by
+// all NT threads; ends without a trailing barrier.
 template <int M, int NT>
 __device__ __forceinline__ void route_staged(const uint4 *rows, int u0, int nu, float tau, uint8_t *sflag,
-                                             uint8_t *mask_out)
+                                             uint8_t *mask_out, float *cosbuf)
 {
     const uint4 *kr = rows + nu * M * 16;
     const int pairs = nu * M;
-    for (int base = 0; base < pairs; base += NT) {
-        const int pr = base + (int)threadIdx.x;
+    const int hw = (int)threadIdx.x >> 4, l16 = (int)threadIdx.x & 15;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int base = 0; base < pairs; base += NT / 16) {
+        const int pr = base + hw;
         const bool valid = pr < pairs;
-        const int lu = pr / M;
-        float c = INFINITY;
-        if (valid)
-            c = head_cosine_smem(rows + pr * 16, kr + lu * 16, (u0 * M + pr) & 15);
-        c = group_min<M>(c);
-        if (valid && pr - lu * M == 0) {
-            const uint8_t sink = (c >= tau) ? 1 : 0;
-            sflag[u0 + lu] = sink;
-            if (mask_out)
-                mask_out[u0 + lu] = sink;
-        }
+        const uint4 qv = valid ? rows[pr * 16 + l16] : zero;
+        const uint4 kv = valid ? kr[(pr / M) * 16 + l16] : zero;
+        const float c = pair_cosine(qv, kv);
+        if (valid && l16 == 0)
+            cosbuf[pr] = c;
+    }
+    __syncthreads();
+    for (int lu = (int)threadIdx.x; lu < nu; lu += NT) {
+        float s = INFINITY;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            s = fminf(s, cosbuf[lu * M + m]);
+        const uint8_t sink = (s >= tau) ? 1 : 0;
+        sflag[u0 + lu] = sink;
+        if (mask_out)
+            mask_out[u0 + lu] = sink;
     }
 }
 
