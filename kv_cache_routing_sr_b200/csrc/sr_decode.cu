@@ -155,6 +155,15 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
 }
 
+// a / b for 0 <= a, 0 < b: 32-bit division when both fit (every workload here),
+// else the 64-bit routine.
+__device__ __forceinline__ long long div_nonneg(long long a, long long b)
+{
+    if (((unsigned long long)a | (unsigned long long)b) <= 0xffffffffull)
+        return (long long)((unsigned)a / (unsigned)b);
+    return a / b;
+}
+
 // Sequence length of unit u, clamped to [1, Lmax] (the prologue reports the
 // clamp; every later lookup must give the same value), from the shared table
 // when the batch fits it.
@@ -417,7 +426,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const int G = gridDim.x;
     long long chunk = 1, r0 = 0, r1 = 0;
     if (p.n_splits == 0 && P > 0) {
-        chunk = (P + G - 1) / G;
+        chunk = div_nonneg(P + G - 1, G);
         chunk = (chunk + C::BN - 1) / C::BN * C::BN;
         chunk = chunk < kMinChunk ? kMinChunk : chunk;
         r0 = (long long)blockIdx.x * chunk;
@@ -536,7 +545,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     const int L = unit_len(p, u, seq_smem ? seqtab : nullptr);
                     const long long b0 = (r0 > S ? r0 : S) - S;
                     const long long e0 = (r1 < S + L ? r1 : S + L) - S;
-                    const long long cf = S / chunk, cl = (S + L - 1) / chunk;
+                    const long long cf = div_nonneg(S, chunk), cl = div_nonneg(S + L - 1, chunk);
                     ok = emit_split(u, b0, e0, (int)blockIdx.x + i, (int)(cl - cf + 1), (int)cf + i);
                     S += L;
                     ++i;
@@ -545,7 +554,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         } else {
             const int ns = p.n_splits;
             for (long long j = blockIdx.x; ok && j < (long long)n * ns; j += G) {
-                const int i = (int)(j / ns), s = (int)(j % ns);
+                const int i = (int)div_nonneg(j, ns), s = (int)(j - (long long)i * ns);
                 const int u = unit_at(i);
                 if (u < 0 || u >= U)
                     break;

@@ -63,8 +63,8 @@ __device__ __forceinline__ float pair_cosine(const uint4 &qv, const uint4 &kv)
 
 // Route the nu units u0 .. u0+nu-1 whose rows are staged in shared memory:
 // `rows` holds their nu*M query rows (row u*M+m of q) followed by their nu key
-// rows, 256 bytes each. NT threads (a multiple of 32) take NT/16 pairs per
-// pass, one per half-warp; the pairs' cosines go to cosbuf (nu*M floats), and
+// rows, 256 bytes each. NT threads (a multiple of 32) take NT/8 pairs per
+// pass, two per half-warp; the pairs' cosines go to cosbuf (nu*M floats), and
 // after a block barrier one thread per unit takes the minimum over its M heads.
 // Writes sflag[u] = sink, and mask_out[u] when mask_out is not null. Called by
 // all NT threads; ends without a trailing barrier.
@@ -76,14 +76,23 @@ __device__ __forceinline__ void route_staged(const uint4 *rows, int u0, int nu, 
     const int pairs = nu * M;
     const int hw = (int)threadIdx.x >> 4, l16 = (int)threadIdx.x & 15;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int base = 0; base < pairs; base += NT / 16) {
-        const int pr = base + hw;
-        const bool valid = pr < pairs;
-        const uint4 qv = valid ? rows[pr * 16 + l16] : zero;
-        const uint4 kv = valid ? kr[(pr / M) * 16 + l16] : zero;
-        const float c = pair_cosine(qv, kv);
-        if (valid && l16 == 0)
-            cosbuf[pr] = c;
+    // Two pairs per half-warp and pass: their loads and shuffle chains are
+    // independent, so they overlap (each pair's arithmetic is unchanged).
+    for (int base = 0; base < pairs; base += NT / 8) {
+        const int pa = base + hw, pb = base + NT / 16 + hw;
+        const bool va = pa < pairs, vb = pb < pairs;
+        const uint4 qa = va ? rows[pa * 16 + l16] : zero;
+        const uint4 ka = va ? kr[(pa / M) * 16 + l16] : zero;
+        const uint4 qb = vb ? rows[pb * 16 + l16] : zero;
+        const uint4 kb = vb ? kr[(pb / M) * 16 + l16] : zero;
+        const float ca = pair_cosine(qa, ka);
+        const float cb = pair_cosine(qb, kb);
+        if (l16 == 0) {
+            if (va)
+                cosbuf[pa] = ca;
+            if (vb)
+                cosbuf[pb] = cb;
+        }
     }
     __syncthreads();
     for (int lu = (int)threadIdx.x; lu < nu; lu += NT) {
