@@ -82,9 +82,10 @@ class ContextParallelDecoder:
     rank's [B, Hkv, shard_max_len, 128] caches and shard_lens [B] int32 (device)
     the lengths of its shards; q, k0, v0 and tau are the same on every rank."""
 
-    def __init__(self, batch, n_q_heads, n_kv_heads, shard_max_len, world: int = 1, group=None, device="cuda"):
+    def __init__(self, batch, n_q_heads, n_kv_heads, shard_max_len, world: int = 1, group=None, device="cuda",
+                 max_splits: int = 0):
         self.B, self.Hq, self.world, self.group = batch, n_q_heads, world, group
-        self.dec = native.Decoder(batch, n_q_heads, n_kv_heads, shard_max_len, device=device)
+        self.dec = native.Decoder(batch, n_q_heads, n_kv_heads, shard_max_len, max_splits=max_splits, device=device)
         self.stride = row_floats(batch, n_q_heads)
         self.gathered = torch.zeros(world * self.stride, dtype=torch.float32, device=device)
         self.row = self.gathered[:self.stride] if world == 1 else torch.zeros(self.stride, dtype=torch.float32,
@@ -131,7 +132,7 @@ def emulate(q, k_cache, v_cache, k0, v0, seq_lens, tau, world: int, n_splits: in
         lens = torch.tensor([e - s for s, e in bounds[r]], dtype=torch.int32, device=q.device)
         shards.append((shard_cache(k_cache, bounds[r]), shard_cache(v_cache, bounds[r]), lens))
     smax = max(k.shape[2] for k, _, _ in shards)
-    cp = ContextParallelDecoder(B, Hq, Hkv, smax, world=1, device=q.device)
+    cp = ContextParallelDecoder(B, Hq, Hkv, smax, world=1, device=q.device, max_splits=n_splits)
     # one rank's decoder, rows for all ranks: the gathered buffer is filled in place
     cp.world = world
     cp.gathered = torch.zeros(world * cp.stride, dtype=torch.float32, device=q.device)

@@ -94,19 +94,21 @@ def test_combine_rejects_bad_layouts():
         native.combine_partials(buf, buf[4096:], 4128, 0, 1, 32)  # no part
 
 
-@pytest.mark.parametrize("name,kw,R", [("llama8b_128k", dict(max_ctx=3000), 2),
-                                       ("llama8b_128k", dict(max_ctx=3000), 8),
-                                       ("llama70b_ragged", dict(max_ctx=2500), 3),
-                                       ("llava7b_mha", dict(max_ctx=1200, batch=3), 5),
-                                       ("tiny_4k", {}, 1)])
-def test_emulated_context_parallel_matches_oracle(name, kw, R):
+@pytest.mark.parametrize("name,kw,R,ns", [("llama8b_128k", dict(max_ctx=3000), 2, 0),
+                                          ("llama8b_128k", dict(max_ctx=3000), 8, 0),
+                                          ("llama70b_ragged", dict(max_ctx=2500), 3, 0),
+                                          ("llava7b_mha", dict(max_ctx=1200, batch=3), 5, 0),
+                                          ("tiny_4k", {}, 1, 0),
+                                          ("llama8b_128k", dict(max_ctx=3000), 4, 7),
+                                          ("llama70b_ragged", dict(max_ctx=2500), 2, 3)])
+def test_emulated_context_parallel_matches_oracle(name, kw, R, ns):
     x = inputs.make(name, seed=5, device=DEV, **kw)
-    out, dec = cp.emulate(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau, R)
+    out, dec = cp.emulate(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau, R, n_splits=ns)
     torch.cuda.synchronize()
     assert dec.dec.workspace.device_error() == 0
     ref = H.oracle_full(x, x.tau)
     H.assert_route_equal(dec.dec.route_mask.cpu(), dec.dec.active_list.cpu(), ref.mask, ref.active_list)
-    H.check_against_oracle(x, out.cpu(), dec.dec.route_mask.cpu(), what=f"{name} R={R}")
+    H.check_against_oracle(x, out.cpu(), dec.dec.route_mask.cpu(), what=f"{name} R={R} n_splits={ns}")
 
 
 def test_emulated_context_parallel_512k_sampled():
