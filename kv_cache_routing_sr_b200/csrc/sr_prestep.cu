@@ -146,6 +146,12 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
         for (int it = threadIdx.x; it < nu * 8; it += kThreads) {
             const int lu = it >> 3, j = it & 7;
             const int u = u0 + lu;
+            // The new key and value do not depend on the slot: load them in the
+            // same round trip as the slot itself.
+            const uint4 *kn = reinterpret_cast<const uint4 *>(p.k_new + (size_t)u * kHeadDim);
+            const uint4 *vn = reinterpret_cast<const uint4 *>(p.v_new + (size_t)u * kHeadDim);
+            const uint4 klo = __ldg(kn + j), khi = __ldg(kn + j + 8);
+            const uint4 vlo = __ldg(vn + j), vhi = __ldg(vn + j + 8);
             const int pos = slot_of(p, u / p.Hkv);
             uint4 *ks = krows + lu * 16;
             uint4 *k0g = reinterpret_cast<uint4 *>(p.k0 + (size_t)u * kHeadDim);
@@ -158,11 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
             float4 c[2], s[2];
             load_table8(p.rope_cos, pos, j, c);
             load_table8(p.rope_sin, pos, j, s);
-            const uint4 *kn = reinterpret_cast<const uint4 *>(p.k_new + (size_t)u * kHeadDim);
-            const uint4 *vn = reinterpret_cast<const uint4 *>(p.v_new + (size_t)u * kHeadDim);
             uint4 lo, hi;
-            rope8(__ldg(kn + j), __ldg(kn + j + 8), c, s, lo, hi);
-            const uint4 vlo = __ldg(vn + j), vhi = __ldg(vn + j + 8);
+            rope8(klo, khi, c, s, lo, hi);
             const size_t slot = ((size_t)u * p.Lmax + pos) * kHeadDim;
             uint4 *kd = reinterpret_cast<uint4 *>(p.k_cache + slot);
             uint4 *vd = reinterpret_cast<uint4 *>(p.v_cache + slot);
@@ -188,8 +191,11 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
         for (int it = threadIdx.x; it < nu * M * 8; it += kThreads) {
             const int r = it >> 3, j = it & 7;
             const int u = u0 + r / M;
-            const int pos = slot_of(p, u / p.Hkv);
             const size_t row = ((size_t)u0 * M + r) * kHeadDim;
+            // plain loads: q_out may be q_in (rotated in place)
+            const uint4 *qi = reinterpret_cast<const uint4 *>(p.q_in + row);
+            const uint4 qlo = qi[j], qhi = qi[j + 8];
+            const int pos = slot_of(p, u / p.Hkv);
             uint4 *qs = rows + r * 16;
             uint4 *qd = reinterpret_cast<uint4 *>(p.q_out + row);
             uint4 lo = zero, hi = zero;
@@ -197,8 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
                 float4 c[2], s[2];
                 load_table8(p.rope_cos, pos, j, c);
                 load_table8(p.rope_sin, pos, j, s);
-                const uint4 *qi = reinterpret_cast<const uint4 *>(p.q_in + row);
-                rope8(qi[j], qi[j + 8], c, s, lo, hi);
+                rope8(qlo, qhi, c, s, lo, hi);
             }
             qs[j] = lo;
             qs[j + 8] = hi;

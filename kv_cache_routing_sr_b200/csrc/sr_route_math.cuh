@@ -114,14 +114,27 @@ namespace sr {
 // Ordered compaction: active[0] = number of units u < U with sflag[u] == 0,
 // active[1..] = those units in ascending order. Warp ballots give each lane's
 // rank inside its warp and a one-warp scan of the per-warp counts gives the
-// warp offsets, NT threads at a time. Called by all NT threads of the block;
-// warp_cnt / warp_off are shared arrays of NT/32 and NT/32 + 1 entries.
+// warp offsets, NT threads at a time (one warp alone when U <= 32). Called by
+// all NT threads of the block after the flags are visible to them (a block
+// barrier); warp_cnt / warp_off are shared arrays of NT/32 and NT/32 + 1 entries.
 template <int NT>
 __device__ __forceinline__ void compact_active(const uint8_t *sflag, int U, int32_t *active, int32_t *warp_cnt,
                                                int32_t *warp_off)
 {
     constexpr int kWarps = NT / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (U <= 32) {
+        // One warp's ballot orders everything; no block barrier needed.
+        if (warp == 0) {
+            const bool act = lane < U && !sflag[lane];
+            const unsigned ball = __ballot_sync(0xffffffffu, act);
+            if (act)
+                active[1 + __popc(ball & ((1u << lane) - 1u))] = lane;
+            if (lane == 0)
+                active[0] = __popc(ball);
+        }
+        return;
+    }
     int32_t total = 0;
     for (int c0 = 0; c0 < U; c0 += NT) {
         const int u = c0 + (int)threadIdx.x;
