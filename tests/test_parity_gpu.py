@@ -127,6 +127,29 @@ def test_decode_full_size_sampled(name):
     H.check_against_oracle(x, out_g, mask_g, units=_sample(mask_g), what=name)
 
 
+@pytest.mark.parametrize("name", ["llama8b_128k", "llama70b_ragged", "llava7b_mha"])
+def test_decode_full_size_every_unit(name):
+    """Every unit of the full-size workload against the oracle (run once on the
+    whole problem, 8 threads): sink heads bit-exact v0, active heads within
+    the tolerances, per (sequence, head)."""
+    x = inputs.make(name, seed=21, device=DEV)
+    mask_g, act_g, out_g, _ = H.gpu_step(x)
+    ref = H.oracle_full(x, x.tau, n_threads=8)
+    H.assert_route_equal(mask_g, act_g, ref.mask, ref.active_list)
+    Hkv, M = x.n_kv_heads, x.n_q_heads // x.n_kv_heads
+    v0 = x.v0.cpu()
+    act = []
+    for u in range(x.batch * Hkv):
+        b, g = divmod(u, Hkv)
+        if mask_g[u]:
+            H.assert_sink_exact(out_g[b, g * M:(g + 1) * M], v0[b, g])
+        else:
+            act.append((b, g))
+    got = torch.stack([out_g[b, g * M:(g + 1) * M] for b, g in act])
+    want = torch.stack([ref.out[b, g * M:(g + 1) * M] for b, g in act])
+    H.assert_active_close(got, want, f"{name}, all {len(act)} active units")
+
+
 @pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
 def test_512k_sink_sweep_sampled(frac):
     x = inputs.make("llama8b_512k", seed=3, device=DEV, sink_fraction=frac)
