@@ -133,35 +133,37 @@ class Oracle:
             raise ValueError(f"sr_oracle_decode failed with status {st}")
         return out, p0
 
+    def rope_append(self, q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache, v_cache, k0, v0):
+        """The step before the scan, on CPU copies of the inputs: RoPE of q and
+        of the new key at slot seq_lens[b], the append, the position-0 capture
+        and the length update. q_in [B,Hq,d], k_new / v_new [B,Hkv,d] (bf16);
+        rope_cos / rope_sin fp32 [max_pos, d/2]; seq_lens int32 [B]; caches
+        [B,Hkv,Lmax,d], k0 / v0 [B,Hkv,d] (bf16). Returns (status, q_out, k_cache,
+        v_cache, k0, v0, seq_lens): status 0 = ok, 1 = some slot out of range
+        (that sequence untouched, its q_out rows zero)."""
+        B, Hq, d = q_in.shape
+        Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+        max_pos = rope_cos.shape[0]
+        kc = k_cache.detach().to("cpu").contiguous().clone()
+        vc = v_cache.detach().to("cpu").contiguous().clone()
+        k0c = k0.detach().to("cpu").contiguous().clone()
+        v0c = v0.detach().to("cpu").contiguous().clone()
+        sl = seq_lens.detach().to("cpu", torch.int32).contiguous().clone()
+        q_out = torch.empty((B, Hq, d), dtype=torch.bfloat16)
+        cs = rope_cos.detach().to("cpu", torch.float32).contiguous()
+        sn = rope_sin.detach().to("cpu", torch.float32).contiguous()
+        qv, qp = self._bits(q_in)
+        kv, kp = self._bits(k_new)
+        vv, vp = self._bits(v_new)
 
-def _rope_append(o: "Oracle", q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache, v_cache, k0, v0):
-    """See Oracle.rope_append."""
-    B, Hq, d = q_in.shape
-    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
-    max_pos = rope_cos.shape[0]
-    kc = k_cache.detach().to("cpu").contiguous().clone()
-    vc = v_cache.detach().to("cpu").contiguous().clone()
-    k0c = k0.detach().to("cpu").contiguous().clone()
-    v0c = v0.detach().to("cpu").contiguous().clone()
-    sl = seq_lens.detach().to("cpu", torch.int32).contiguous().clone()
-    q_out = torch.empty((B, Hq, d), dtype=torch.bfloat16)
-    cs = rope_cos.detach().to("cpu", torch.float32).contiguous()
-    sn = rope_sin.detach().to("cpu", torch.float32).contiguous()
-    qv, qp = o._bits(q_in)
-    kv_, kp = o._bits(k_new)
-    vv_, vp = o._bits(v_new)
-    u16 = lambda t: ctypes.cast(t.view(torch.int16).data_ptr(), ctypes.POINTER(ctypes.c_uint16))  # noqa: E731
-    st = o._lib.sr_oracle_rope_append(B, Hq, Hkv, d, Lmax, max_pos, qp, kp, vp, o._ptr(cs, ctypes.c_float),
-                                      o._ptr(sn, ctypes.c_float), o._ptr(sl, ctypes.c_int32), u16(kc), u16(vc),
-                                      u16(k0c), u16(v0c), u16(q_out))
-    return st, q_out, kc, vc, k0c, v0c, sl
+        def u16(t):
+            return ctypes.cast(t.view(torch.int16).data_ptr(), ctypes.POINTER(ctypes.c_uint16))
 
-
-Oracle.rope_append = lambda self, *a: _rope_append(self, *a)
-Oracle.rope_append.__doc__ = """The step before the scan on CPU copies: returns (status, q_out, k_cache,
-v_cache, k0, v0, seq_lens) after RoPE of q and of the new key at slot
-seq_lens[b], the append, the position-0 capture and the length update.
-status 0 = ok, 1 = some slot out of range (that sequence untouched)."""
+        st = self._lib.sr_oracle_rope_append(B, Hq, Hkv, d, Lmax, max_pos, qp, kp, vp,
+                                             self._ptr(cs, ctypes.c_float), self._ptr(sn, ctypes.c_float),
+                                             self._ptr(sl, ctypes.c_int32), u16(kc), u16(vc), u16(k0c), u16(v0c),
+                                             u16(q_out))
+        return st, q_out, kc, vc, k0c, v0c, sl
 
 
 @dataclass
