@@ -650,12 +650,17 @@ def run_ours(args):
         line["sweep_512k"] = sweep
     if world == 1 and not args.no_sweep:
         # The remaining workloads: tiny 4K with L2 hot and cold (rotating over
-        # input sets that together exceed L2), the ragged 70B-shaped and the
+        # input sets that together exceed L2), the 128K layer rotating over
+        # three input sets instead of flushing, the ragged 70B-shaped and the
         # LLaVA-shaped layers with the flush protocol.
         oc_steps = max(20, min(K, 50))
         line["other_configs"] = [
             measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "hot"),
             measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "rotate", copies=12),
+            # the headline workload with the other valid L2 protocol: three
+            # independent layer inputs in rotation, each step streaming 268 MB
+            measure_config(native, inputs, "llama8b_128k", oc_steps, args.warmup, flush, dev, peak, "rotate",
+                           copies=3),
             measure_config(native, inputs, "llama70b_ragged", oc_steps, args.warmup, flush, dev, peak),
             measure_config(native, inputs, "llava7b_mha", oc_steps, args.warmup, flush, dev, peak),
         ]
