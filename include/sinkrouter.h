@@ -291,6 +291,21 @@ sr_status sr_decode_attention_partial(const sr_dims *dims, const void *q, const 
 sr_status sr_combine_partials(const sr_dims *dims, int32_t n_parts, const float *o_parts,
                               const float *lse_parts, int64_t part_stride, void *out, void *stream);
 
+/*
+ * sr_selftest_bounded_wait -- exercise the time-bounded wait that every kernel
+ * of this library uses instead of an unbounded spin: one warp waits on an
+ * mbarrier that nothing ever arrives on, gives up after limit_us microseconds
+ * (read from %globaltimer) and reports it. (An engineering self-test; the
+ * pages have no counterpart.)
+ *   limit_us   1 .. 2000000 (the kernels' own bound is 2 s)
+ *   status     out device int32: SR_DEVERR_TIMEOUT when the wait ran out (the
+ *              expected result), 0 if it completed
+ *   waited_ns  out device uint64: how long the warp waited
+ * One launch of one warp on `stream`; the context stays usable afterwards.
+ * Errors: SR_ERR_INVALID_ARG, SR_ERR_CUDA.
+ */
+sr_status sr_selftest_bounded_wait(int32_t limit_us, int32_t *status, uint64_t *waited_ns, void *stream);
+
 /* Static description of a status code. */
 const char *sr_status_string(sr_status s);
 

@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libsinkrouter.so")
-SOURCES = ["sr_abi.cu", "sr_route.cu", "sr_prestep.cu", "sr_decode.cu", "sr_combine.cu", "sr_static_scratch.cu"]
+SOURCES = ["sr_abi.cu", "sr_route.cu", "sr_prestep.cu", "sr_decode.cu", "sr_combine.cu", "sr_static_scratch.cu",
+           "sr_selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

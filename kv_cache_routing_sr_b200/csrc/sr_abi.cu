@@ -258,6 +258,15 @@ sr_status sr_combine_partials(const sr_dims *dims, int32_t n_parts, const float 
     return e == cudaSuccess ? SR_OK : cuda_fail(e);
 }
 
+sr_status sr_selftest_bounded_wait(int32_t limit_us, int32_t *status, uint64_t *waited_ns, void *stream)
+{
+    if (limit_us < 1 || limit_us > 2000000 || !status || !aligned(status, 4) || !waited_ns || !aligned(waited_ns, 8))
+        return SR_ERR_INVALID_ARG;
+    const cudaError_t e = sr::launch_bounded_wait_selftest(
+        limit_us, status, reinterpret_cast<unsigned long long *>(waited_ns), as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
 sr_status sr_route_decode_attention(const sr_dims *dims, const void *q, const void *k_cache, const void *v_cache,
                                     const void *k0, const void *v0, const int32_t *seq_lens, float tau,
                                     int32_t n_splits, uint8_t *route_mask, int32_t *active_list, void *out,

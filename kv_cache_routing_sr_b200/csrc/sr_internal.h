@@ -87,6 +87,9 @@ struct PrestepArgs {
 
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);
 cudaError_t launch_rope_append_route(const PrestepArgs &a, cudaStream_t stream);
+// Self-test of the bounded wait (sr_selftest_bounded_wait).
+cudaError_t launch_bounded_wait_selftest(int32_t limit_us, int32_t *status, unsigned long long *waited_ns,
+                                         cudaStream_t stream);
 // Log-sum-exp combination of n_parts partial outputs (sr_combine_partials).
 cudaError_t launch_combine(int n_heads, int n_parts, const float *o_parts, const float *lse_parts, int64_t part_stride,
                            void *out, cudaStream_t stream);

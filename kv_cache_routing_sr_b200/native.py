@@ -42,7 +42,7 @@ EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_dec
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
            "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention",
            "sr_decode_attention_lse", "sr_rope_append_route", "sr_decode_attention_partial",
-           "sr_combine_partials"]
+           "sr_combine_partials", "sr_selftest_bounded_wait"]
 
 
 def load(path: str = LIBRARY):
@@ -88,6 +88,8 @@ def load(path: str = LIBRARY):
     lib.sr_decode_attention_partial.restype = ctypes.c_int
     lib.sr_combine_partials.argtypes = [dp, i32, vp, vp, ctypes.c_int64, vp, vp]
     lib.sr_combine_partials.restype = ctypes.c_int
+    lib.sr_selftest_bounded_wait.argtypes = [i32, vp, vp, vp]
+    lib.sr_selftest_bounded_wait.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -306,6 +308,19 @@ def rope_append_route(q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache,
         _dev(active_list, "active_list", torch.int32), err or None, _stream(stream))
     _check("sr_rope_append_route", st)
     return q_out, route_mask, active_list
+
+
+def selftest_bounded_wait(limit_us: int, device="cuda", stream=None):
+    """sr_selftest_bounded_wait: a wait on an mbarrier nothing arrives on, with
+    a bound of limit_us. Returns (status, waited_ns) after synchronising; the
+    expected status is SR_DEVERR_TIMEOUT."""
+    status = torch.full((1,), -1, dtype=torch.int32, device=device)
+    waited = torch.zeros(1, dtype=torch.int64, device=device)
+    _check("sr_selftest_bounded_wait",
+           load().sr_selftest_bounded_wait(int(limit_us), _dev(status, "status", torch.int32),
+                                           _dev(waited, "waited_ns", torch.int64), _stream(stream)))
+    torch.cuda.synchronize(device)
+    return int(status.item()), int(waited.item())
 
 
 def grid_size() -> int:

@@ -148,3 +148,14 @@ def test_rope_append_route_validation(lib):
     assert c(max_pos=0) == native.SR_ERR_INVALID_ARG
     assert c(tau=float("nan")) == native.SR_ERR_INVALID_ARG
     assert c(dims=dims(d=64)) == native.SR_ERR_UNSUPPORTED
+
+
+def test_bounded_wait_selftest_validation(lib):
+    """Host-side refusals of sr_selftest_bounded_wait: nothing is launched."""
+    c = lambda lim, st=FAKE, w=FAKE: lib.sr_selftest_bounded_wait(lim, st, w, None)  # noqa: E731
+    assert c(0) == native.SR_ERR_INVALID_ARG
+    assert c(2000001) == native.SR_ERR_INVALID_ARG
+    assert c(1000, st=None) == native.SR_ERR_INVALID_ARG
+    assert c(1000, st=FAKE + 2) == native.SR_ERR_INVALID_ARG
+    assert c(1000, w=None) == native.SR_ERR_INVALID_ARG
+    assert c(1000, w=FAKE + 4) == native.SR_ERR_INVALID_ARG
