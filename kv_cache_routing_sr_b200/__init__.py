@@ -7,7 +7,7 @@ call into ``native`` does, and raises if it is missing or cannot run.
 """
 from importlib import import_module
 
-__all__ = ["native", "inputs", "multilayer"]
+__all__ = ["native", "inputs", "multilayer", "context_parallel", "proxy_quality", "build"]
 
 
 def __getattr__(name):

@@ -132,10 +132,9 @@ def emulate(q, k_cache, v_cache, k0, v0, seq_lens, tau, world: int, n_splits: in
         lens = torch.tensor([e - s for s, e in bounds[r]], dtype=torch.int32, device=q.device)
         shards.append((shard_cache(k_cache, bounds[r]), shard_cache(v_cache, bounds[r]), lens))
     smax = max(k.shape[2] for k, _, _ in shards)
-    cp = ContextParallelDecoder(B, Hq, Hkv, smax, world=1, device=q.device, max_splits=n_splits)
-    # one rank's decoder, rows for all ranks: the gathered buffer is filled in place
-    cp.world = world
-    cp.gathered = torch.zeros(world * cp.stride, dtype=torch.float32, device=q.device)
+    # one decoder with every rank's row: each shard's scan writes its row of the
+    # gathered buffer in place, so the exchange (finish) is never needed
+    cp = ContextParallelDecoder(B, Hq, Hkv, smax, world=world, device=q.device, max_splits=n_splits)
     for r, (ks, vs, lens) in enumerate(shards):
         cp.local(q, ks, vs, k0, v0, lens, tau, n_splits, row=cp.gathered[r * cp.stride:(r + 1) * cp.stride])
     n = B * Hq

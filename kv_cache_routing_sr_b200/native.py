@@ -7,6 +7,7 @@ CPU fallback: a missing or unloadable library raises.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -94,6 +95,17 @@ def load(path: str = LIBRARY):
     return lib
 
 
+def _on_tensor_device(fn):
+    """Run fn with the device of its first (tensor) argument current: the
+    library launches on the current device, and the default stream passed to it
+    must be that device's."""
+    @functools.wraps(fn)
+    def wrapper(t, *args, **kwargs):
+        with torch.cuda.device(t.device):
+            return fn(t, *args, **kwargs)
+    return wrapper
+
+
 def _check(fn: str, status: int):
     if status != SR_OK:
         raise SinkRouterError(fn, status, load())
@@ -134,8 +146,9 @@ class Workspace:
         self.buffer = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
         off = (-self.buffer.data_ptr()) % 256
         self.view = self.buffer[off:off + self.nbytes]
-        _check("sr_workspace_init", load().sr_workspace_init(ctypes.c_void_p(self.view.data_ptr()),
-                                                             self.nbytes, _stream()))
+        with torch.cuda.device(self.buffer.device):
+            _check("sr_workspace_init", load().sr_workspace_init(ctypes.c_void_p(self.view.data_ptr()),
+                                                                 self.nbytes, _stream()))
 
     @property
     def ptr(self) -> int:
@@ -143,14 +156,17 @@ class Workspace:
 
     def device_error(self) -> int:
         code = ctypes.c_int32(0)
-        _check("sr_get_device_error", load().sr_get_device_error(ctypes.c_void_p(self.ptr),
-                                                                 ctypes.byref(code), _stream()))
+        with torch.cuda.device(self.buffer.device):
+            _check("sr_get_device_error", load().sr_get_device_error(ctypes.c_void_p(self.ptr),
+                                                                     ctypes.byref(code), _stream()))
         return int(code.value)
 
     def clear_device_error(self):
-        _check("sr_clear_device_error", load().sr_clear_device_error(ctypes.c_void_p(self.ptr), _stream()))
+        with torch.cuda.device(self.buffer.device):
+            _check("sr_clear_device_error", load().sr_clear_device_error(ctypes.c_void_p(self.ptr), _stream()))
 
 
+@_on_tensor_device
 def route(q: torch.Tensor, k0: torch.Tensor, tau: float, route_mask=None, active_list=None, stream=None):
     """sr_route: returns (route_mask uint8 [B*Hkv], active_list int32 [1+B*Hkv])."""
     B, Hq, d = q.shape
@@ -167,6 +183,7 @@ def route(q: torch.Tensor, k0: torch.Tensor, tau: float, route_mask=None, active
     return route_mask, active_list
 
 
+@_on_tensor_device
 def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=None, n_splits: int = 0,
                      workspace: Workspace | None = None, stream=None, lse=None):
     """sr_decode_attention: returns out bf16 [B, Hq, 128]. With ``lse`` (an fp32
@@ -193,6 +210,7 @@ def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=Non
     return out
 
 
+@_on_tensor_device
 def decode_attention_partial(q, k_cache, v_cache, k0, v0, seq_lens, active_list, o_part=None, lse_part=None,
                              n_splits: int = 0, workspace: Workspace | None = None, stream=None):
     """sr_decode_attention_partial: the scan over this cache's positions with
@@ -218,6 +236,7 @@ def decode_attention_partial(q, k_cache, v_cache, k0, v0, seq_lens, active_list,
     return o_part, lse_part
 
 
+@_on_tensor_device
 def combine_partials(o_parts, lse_parts, part_stride: int, n_parts: int, batch: int, n_q_heads: int, out=None,
                      stream=None):
     """sr_combine_partials over n_parts parts laid out part_stride floats apart:
@@ -235,6 +254,7 @@ def combine_partials(o_parts, lse_parts, part_stride: int, n_parts: int, batch: 
     return out
 
 
+@_on_tensor_device
 def decode_attention_static_scratch(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=None,
                                     n_splits: int = 0, device_error=None, stream=None):
     """sr_decode_attention_static_scratch: the decode step with the library's
@@ -257,6 +277,7 @@ def decode_attention_static_scratch(q, k_cache, v_cache, k0, v0, seq_lens, activ
     return out
 
 
+@_on_tensor_device
 def route_decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, tau, out=None, route_mask=None,
                            active_list=None, n_splits: int = 0, workspace: Workspace | None = None, stream=None):
     """sr_route_decode_attention: routing and decode in one launch. Returns out;
@@ -279,6 +300,7 @@ def route_decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, tau, out=None,
     return out
 
 
+@_on_tensor_device
 def rope_append_route(q_in, k_new, v_new, rope_cos, rope_sin, seq_lens, k_cache, v_cache, k0, v0, tau,
                       q_out=None, route_mask=None, active_list=None, device_error=None, stream=None):
     """sr_rope_append_route: RoPE of the query and the new key at slot
@@ -316,9 +338,10 @@ def selftest_bounded_wait(limit_us: int, device="cuda", stream=None):
     expected status is SR_DEVERR_TIMEOUT."""
     status = torch.full((1,), -1, dtype=torch.int32, device=device)
     waited = torch.zeros(1, dtype=torch.int64, device=device)
-    _check("sr_selftest_bounded_wait",
-           load().sr_selftest_bounded_wait(int(limit_us), _dev(status, "status", torch.int32),
-                                           _dev(waited, "waited_ns", torch.int64), _stream(stream)))
+    with torch.cuda.device(status.device):
+        _check("sr_selftest_bounded_wait",
+               load().sr_selftest_bounded_wait(int(limit_us), _dev(status, "status", torch.int32),
+                                               _dev(waited, "waited_ns", torch.int64), _stream(stream)))
     torch.cuda.synchronize(device)
     return int(status.item()), int(waited.item())
 
