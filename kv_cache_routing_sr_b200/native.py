@@ -139,7 +139,8 @@ def workspace_bytes(batch, n_q_heads, n_kv_heads, max_seq_len, max_splits: int =
 
 
 class Workspace:
-    """A zero-initialised decode workspace in torch-allocated device memory."""
+    """A zero-initialised decode workspace in torch-allocated device memory,
+    usable from any stream once constructed."""
 
     def __init__(self, batch, n_q_heads, n_kv_heads, max_seq_len, max_splits: int = 0, device=None):
         self.nbytes = workspace_bytes(batch, n_q_heads, n_kv_heads, max_seq_len, max_splits)
@@ -149,6 +150,9 @@ class Workspace:
         with torch.cuda.device(self.buffer.device):
             _check("sr_workspace_init", load().sr_workspace_init(ctypes.c_void_p(self.view.data_ptr()),
                                                                  self.nbytes, _stream()))
+            # the zeroing must be complete before any stream uses the workspace
+            # (side streams do not wait for the stream it was issued on)
+            torch.cuda.current_stream().synchronize()
 
     @property
     def ptr(self) -> int:

@@ -464,3 +464,42 @@ def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
     ref, _ = oracle.decode(q[:1, :M].cpu(), kc[:1, :1].cpu(), vc[:1, :1].cpu(), v0[:1, :1].cpu(),
                            sl[:1].cpu(), torch.zeros(1, dtype=torch.uint8))
     H.assert_active_close(a[0].unsqueeze(0), ref[0].unsqueeze(0), f"M={M} ns={ns}")
+
+
+def test_concurrent_host_threads_on_separate_streams():
+    """Two host threads, each with its own Decoder (workspace, route buffers)
+    and CUDA stream, run decode steps concurrently; every output equals the
+    serial result bit for bit (the library's lazily built per-device state is
+    safe to share)."""
+    import threading
+
+    xs = [inputs.make("llama70b_ragged", seed=70 + i, device=DEV, max_ctx=3000) for i in range(2)]
+    refs = []
+    for x in xs:
+        _, _, out, _ = H.gpu_step(x)
+        refs.append(out.clone())
+    results, errors = [[], []], []
+
+    def worker(i):
+        try:
+            x = xs[i]
+            st = torch.cuda.Stream()
+            dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+            with torch.cuda.stream(st):
+                for _ in range(30):
+                    out = dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau, stream=st)
+                    results[i].append(out.clone())
+            st.synchronize()
+        except Exception as e:  # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    for i in range(2):
+        assert len(results[i]) == 30
+        for out in results[i]:
+            assert torch.equal(out.cpu().view(torch.int16), refs[i].cpu().view(torch.int16))
