@@ -47,10 +47,18 @@ EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_dec
 
 
 def load(path: str = LIBRARY):
-    """Load (once) and type the library. Raises if it is missing."""
+    """Load (once) and type the library. The in-tree library is compiled first
+    if it is absent (nvcc, sm_100a); any other missing path, or a failed
+    compile, raises: there is no other implementation to fall back to."""
     global _lib
     if _lib is not None:
         return _lib
+    if not os.path.exists(path) and os.path.abspath(path) == os.path.abspath(LIBRARY):
+        from . import build as _build
+        try:
+            _build.build()
+        except Exception as e:
+            raise RuntimeError(f"libsinkrouter.so is missing and compiling it failed: {e}") from e
     if not os.path.exists(path):
         raise RuntimeError(f"libsinkrouter.so not found at {path}: build it with "
                            "`python -m kv_cache_routing_sr_b200.build` (nvcc, sm_100a)")
