@@ -470,6 +470,23 @@ def e2e_measure(native, x, steps):
     return ms, h2d, d2h
 
 
+def _packed_token_inputs(a):
+    """The new token's q/k/v projections packed in one pinned host buffer and
+    one device buffer (views of each), so that a step moves them with a single
+    host -> device copy. Returns (host, device, views on the device)."""
+    import torch
+    parts = [a.q_in, a.k_new, a.v_new]
+    sizes = [t.numel() for t in parts]
+    host = torch.empty(sum(sizes), dtype=torch.bfloat16).pin_memory()
+    dev = torch.empty(sum(sizes), dtype=torch.bfloat16, device=a.q_in.device)
+    views, off = [], 0
+    for t, n in zip(parts, sizes):
+        host[off:off + n].copy_(t.reshape(-1).cpu())
+        views.append(dev[off:off + n].view(t.shape))
+        off += n
+    return host, dev, views
+
+
 def e2e_append_measure(native, x, a, steps):
     """The serving view of the same step through the public API: per step only
     the new token's projections (q_in, k_new, v_new) come from pinned host
@@ -478,21 +495,18 @@ def e2e_append_measure(native, x, a, steps):
     seq_lens is restored on the device each step so that the context stays at
     the workload's length."""
     import torch
-    host = {n: getattr(a, n).cpu().pin_memory() for n in ("q_in", "k_new", "v_new")}
-    dev = {n: torch.empty_like(getattr(a, n)) for n in host}
+    host, dev, (q_in, k_new, v_new) = _packed_token_inputs(a)
     dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
     out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
     mask_h = torch.empty(dec.route_mask.shape, dtype=dec.route_mask.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = host.numel() * host.element_size()
     d2h = out_h.numel() * out_h.element_size() + mask_h.numel()
     st = torch.cuda.current_stream()
 
     def one():
-        for n in host:
-            dev[n].copy_(host[n], non_blocking=True)
+        dev.copy_(host, non_blocking=True)
         a.seq_lens.copy_(a.seq_saved)
-        dec.append_step(dev["q_in"], dev["k_new"], dev["v_new"], a.cos, a.sin, x.k_cache, x.v_cache, x.k0, x.v0,
-                        a.seq_lens, x.tau)
+        dec.append_step(q_in, k_new, v_new, a.cos, a.sin, x.k_cache, x.v_cache, x.k0, x.v0, a.seq_lens, x.tau)
         out_h.copy_(dec.out, non_blocking=True)
         mask_h.copy_(dec.route_mask, non_blocking=True)
 
@@ -506,6 +520,46 @@ def e2e_append_measure(native, x, a, steps):
     e1.record(st)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def e2e_append_graph_measure(native, x, a, steps):
+    """e2e_append with the whole step captured in one CUDA graph (the way a
+    decode server replays a layer): per replay the new token's q/k/v copies
+    from pinned host memory, the seq_lens reset, the append step and the scan,
+    and the copies of the output and mask back to pinned host memory."""
+    import torch
+    host, dev, (q_in, k_new, v_new) = _packed_token_inputs(a)
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
+    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    mask_h = torch.empty(dec.route_mask.shape, dtype=dec.route_mask.dtype).pin_memory()
+
+    def one():
+        dev.copy_(host, non_blocking=True)
+        a.seq_lens.copy_(a.seq_saved)
+        dec.append_step(q_in, k_new, v_new, a.cos, a.sin, x.k_cache, x.v_cache, x.k0, x.v0, a.seq_lens, x.tau)
+        out_h.copy_(dec.out, non_blocking=True)
+        mask_h.copy_(dec.route_mask, non_blocking=True)
+
+    side = torch.cuda.Stream(device=x.q.device)
+    side.wait_stream(torch.cuda.current_stream(x.q.device))
+    with torch.cuda.stream(side):
+        one()
+    torch.cuda.current_stream(x.q.device).wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        one()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / steps
 
 
 def oracle_layer_step_us(x_cpu, budget_s, min_reps=1, threads=None):
@@ -676,8 +730,18 @@ def run_ours(args):
         line["e2e_append"] = {"value": round(ms_a * 1e3 / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d_a,
                               "d2h_bytes_per_step": d2h_a,
                               "path": "Decoder.append_step, eager launch, KV cache resident",
-                              "note": "per step: the new token's q/k/v projections host -> device, the output "
-                                      "and route mask device -> host"}
+                              "note": "per step: the new token's q/k/v projections host -> device in one "
+                                      "packed copy, the output and route mask device -> host"}
+        try:
+            ms_g = e2e_append_graph_measure(native, x, app, max(args.e2e_steps, 50))
+            failed = 0.0
+        except Exception as e:  # capture of the host copies refused: report, do not fail the run
+            ms_g, failed, why = 0.0, 1.0, f"{type(e).__name__}: {str(e)[:160]}"
+        ms_g, failed = max_over_ranks(ms_g), max_over_ranks(failed)  # same collectives on every rank
+        line["e2e_append"]["graph_replay"] = (
+            {"value": round(ms_g * 1e3 / world, 3), "unit": UNIT,
+             "note": "the same copies and calls captured in one CUDA graph, one replay per step"}
+            if not failed else {"unavailable": why if "why" in locals() else "failed on another rank"})
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         xc = x.to("cpu")
         us, threads, reps, el = oracle_layer_step_us(xc, args.cpu_budget_s)
