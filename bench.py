@@ -9,10 +9,16 @@ head_dim 128, bf16 cache, 4 of 8 KV groups planted sinks, tau 0.6.
 Prints one JSON line (rank 0): µs per layer-step (lower is better), effective
 HBM GB/s over the bytes the step must move, the roofline of the decode kernel
 against the measured HBM copy bandwidth, the same kernel with routing disabled
-(tau = +inf), the fp64 CPU oracle on this host's cores, an end-to-end figure
-with host buffers, and the SM clocks seen during the timed region.
+(tau = +inf), the fused single launch, the append step (RoPE + KV append +
+routing, then the scan), the 512K sink-fraction sweep and the other workloads
+(one GPU), the fp64 CPU oracle on this host's cores, end-to-end figures with
+host buffers (every input each step; and the serving view, only the new token's
+projections), and the SM clocks seen during the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --multilayer        # per-token latency of a gated 32-layer graph
+    python bench.py --proxy-quality     # routing proxy vs full-attention sink event
+    python bench.py --context-parallel  # one 512K layer-step sharded over the ranks
 
 Multi-GPU (torchrun): every rank runs its own independent layer-step (the
 units of a decode step share nothing); time is the max over ranks and the value
