@@ -219,13 +219,14 @@ typedef struct {
 } oracle_job;
 
 /*
- * One group (steps 2 and 3 above) for every head of the group.
+ * One head m of one group (steps 2 and 3 above).
  * Active path: logits l_j = <q_h, K_j> / sqrt(d) for j = 0 .. L-1 (position 0
  * read from the cache), p = exp(l - max l) / sum, out = sum_j p_j V_j, and the
  * weight p_0 of position 0 is also returned. Sink path: out = v0 exactly and
- * p_0 is reported as NaN (no attention was computed).
+ * p_0 is reported as NaN (no attention was computed). Each head of a group is
+ * computed on its own, so splitting the work by head changes no arithmetic.
  */
-static int oracle_unit(const oracle_job *J, int unit, double *logit)
+static int oracle_head(const oracle_job *J, int unit, int m, double *logit)
 {
     int M = J->Hq / J->Hkv;
     int b = unit / J->Hkv, g = unit % J->Hkv;
@@ -236,44 +237,42 @@ static int oracle_unit(const oracle_job *J, int unit, double *logit)
     const uint16_t *K = J->kc + ((size_t)b * J->Hkv + g) * (size_t)J->Lmax * d;
     const uint16_t *V = J->vc + ((size_t)b * J->Hkv + g) * (size_t)J->Lmax * d;
     double scale = 1.0 / sqrt((double)d);
-    for (int m = 0; m < M; ++m) {
-        int h = g * M + m;
-        double *o = J->out + ((size_t)b * J->Hq + h) * d;
-        if (J->mask[unit]) {
-            const uint16_t *v0g = J->v0 + ((size_t)b * J->Hkv + g) * d;
-            for (int i = 0; i < d; ++i)
-                o[i] = widen_bf16(v0g[i]);
-            if (J->p0)
-                J->p0[(size_t)b * J->Hq + h] = NAN;
-            continue;
-        }
-        const uint16_t *qh = J->q + ((size_t)b * J->Hq + h) * d;
-        double mx = -INFINITY;
-        for (int j = 0; j < L; ++j) {
-            double acc = 0.0;
-            const uint16_t *kj = K + (size_t)j * d;
-            for (int i = 0; i < d; ++i)
-                acc += widen_bf16(qh[i]) * widen_bf16(kj[i]);
-            logit[j] = acc * scale;
-            if (logit[j] > mx)
-                mx = logit[j];
-        }
-        double z = 0.0;
-        for (int j = 0; j < L; ++j) {
-            logit[j] = exp(logit[j] - mx);
-            z += logit[j];
-        }
+    int h = g * M + m;
+    double *o = J->out + ((size_t)b * J->Hq + h) * d;
+    if (J->mask[unit]) {
+        const uint16_t *v0g = J->v0 + ((size_t)b * J->Hkv + g) * d;
         for (int i = 0; i < d; ++i)
-            o[i] = 0.0;
-        for (int j = 0; j < L; ++j) {
-            double p = logit[j] / z;
-            const uint16_t *vj = V + (size_t)j * d;
-            for (int i = 0; i < d; ++i)
-                o[i] += p * widen_bf16(vj[i]);
-        }
+            o[i] = widen_bf16(v0g[i]);
         if (J->p0)
-            J->p0[(size_t)b * J->Hq + h] = logit[0] / z;
+            J->p0[(size_t)b * J->Hq + h] = NAN;
+        return SR_ORACLE_OK;
     }
+    const uint16_t *qh = J->q + ((size_t)b * J->Hq + h) * d;
+    double mx = -INFINITY;
+    for (int j = 0; j < L; ++j) {
+        double acc = 0.0;
+        const uint16_t *kj = K + (size_t)j * d;
+        for (int i = 0; i < d; ++i)
+            acc += widen_bf16(qh[i]) * widen_bf16(kj[i]);
+        logit[j] = acc * scale;
+        if (logit[j] > mx)
+            mx = logit[j];
+    }
+    double z = 0.0;
+    for (int j = 0; j < L; ++j) {
+        logit[j] = exp(logit[j] - mx);
+        z += logit[j];
+    }
+    for (int i = 0; i < d; ++i)
+        o[i] = 0.0;
+    for (int j = 0; j < L; ++j) {
+        double p = logit[j] / z;
+        const uint16_t *vj = V + (size_t)j * d;
+        for (int i = 0; i < d; ++i)
+            o[i] += p * widen_bf16(vj[i]);
+    }
+    if (J->p0)
+        J->p0[(size_t)b * J->Hq + h] = logit[0] / z;
     return SR_ORACLE_OK;
 }
 
@@ -285,8 +284,9 @@ static void *oracle_worker(void *arg)
         J->status = SR_ORACLE_NO_MEM;
         return NULL;
     }
-    for (int k = J->tid; k < J->n_units; k += J->n_threads) {
-        int st = oracle_unit(J, J->units[k], logit);
+    int M = J->Hq / J->Hkv;
+    for (long k = J->tid; k < (long)J->n_units * M; k += J->n_threads) {
+        int st = oracle_head(J, J->units[k / M], (int)(k % M), logit);
         if (st != SR_ORACLE_OK) {
             J->status = st;
             break;
@@ -304,8 +304,9 @@ static void *oracle_worker(void *arg)
  *   units [n_units]: flat group indices to compute; NULL = every group
  *   out [B,Hq,d] fp64 and p0 [B,Hq] fp64 (p0 may be NULL): only the heads of
  *   the listed groups are written
- *   n_threads: worker threads; groups are dealt round-robin, each group is
- *   computed whole by one thread, so the result does not depend on it
+ *   n_threads: worker threads; the (group, head) pairs are dealt round-robin,
+ *   each head is computed whole by one thread, so the result does not depend
+ *   on it
  */
 int sr_oracle_decode(int B, int Hq, int Hkv, int d, int Lmax,
                      const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
@@ -333,8 +334,8 @@ int sr_oracle_decode(int B, int Hq, int Hkv, int d, int Lmax,
         }
     if (n_threads < 1)
         n_threads = 1;
-    if (n_threads > n_units)
-        n_threads = n_units > 0 ? n_units : 1;
+    if ((long)n_threads > (long)n_units * (Hq / Hkv))
+        n_threads = n_units > 0 ? n_units * (Hq / Hkv) : 1;
     oracle_job *jobs = (oracle_job *)calloc((size_t)n_threads, sizeof(oracle_job));
     pthread_t *th = (pthread_t *)calloc((size_t)n_threads, sizeof(pthread_t));
     if (!jobs || !th) {

@@ -12,13 +12,13 @@ from tests import pins
 
 MUTANTS = [
     ("scale_1_over_d", "double scale = 1.0 / sqrt((double)d);", "double scale = 1.0 / (double)d;"),
-    ("interleaved_head_map", "        int h = g * M + m;\n        double *o", "        int h = m * J->Hkv + g;\n        double *o"),
+    ("interleaved_head_map", "    int h = g * M + m;\n    double *o", "    int h = m * J->Hkv + g;\n    double *o"),
     ("drops_position_0",
-     "for (int j = 0; j < L; ++j) {\n            double acc = 0.0;",
-     "for (int j = 1; j < L; ++j) {\n            double acc = 0.0;"),
+     "for (int j = 0; j < L; ++j) {\n        double acc = 0.0;",
+     "for (int j = 1; j < L; ++j) {\n        double acc = 0.0;"),
     ("drops_last_position",
-     "for (int j = 0; j < L; ++j) {\n            double acc = 0.0;",
-     "for (int j = 0; j < L - 1; ++j) {\n            double acc = 0.0;"),
+     "for (int j = 0; j < L; ++j) {\n        double acc = 0.0;",
+     "for (int j = 0; j < L - 1; ++j) {\n        double acc = 0.0;"),
     ("unnormalised_weights", "double p = logit[j] / z;", "double p = logit[j];"),
     ("keys_read_from_values", "const uint16_t *kj = K + (size_t)j * d;", "const uint16_t *kj = V + (size_t)j * d;"),
     ("max_over_heads", "if (c < s)\n                    s = c;", "if (c > s || m == 0)\n                    s = c;"),

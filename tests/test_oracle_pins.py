@@ -15,8 +15,11 @@ def test_thread_count_does_not_change_results(oracle_lib):
     seq[1] = 123
     mask, _, _ = oracle_lib.route(q, k0, 0.6)
     o1, p1 = oracle_lib.decode(q, k, v, v0, seq, mask, n_threads=1)
-    o4, p4 = oracle_lib.decode(q, k, v, v0, seq, mask, n_threads=4)
-    assert torch.equal(o1, o4) and torch.equal(torch.nan_to_num(p1), torch.nan_to_num(p4))
+    # fewer threads than units, between units and (unit, head) pairs, and more
+    # than pairs: the oracle deals whole heads to its threads
+    for nt in (4, 7, 13, 64):
+        o4, p4 = oracle_lib.decode(q, k, v, v0, seq, mask, n_threads=nt)
+        assert torch.equal(o1, o4) and torch.equal(torch.nan_to_num(p1), torch.nan_to_num(p4)), nt
 
 
 def test_unit_subset_matches_full(oracle_lib):
