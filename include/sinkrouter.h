@@ -354,9 +354,10 @@ const char *sr_last_cuda_error(void);
  *     with M = 1);
  *   - device_error: optional device pointer (NULL = not wanted) that receives
  *     the launch's device error word (SR_DEVERR_* bits), stream-ordered;
- *   - the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) and may load the module there; make that first
- *     call before any stream capture;
+ *   - every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, cheap once the module is loaded there), so no
+ *     address survives a device reset; the first call on a device may load
+ *     the module there, so make that first call before any stream capture;
  *   - every call on a device shares the one array: each call clears the error
  *     word and the counters it needs, so calls in sequence on one stream are
  *     fine, but calls that overlap on the GPU (different streams, or host

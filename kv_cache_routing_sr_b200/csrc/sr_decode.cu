@@ -47,6 +47,7 @@
 #include "sr_internal.h"
 #include "sr_ptx.cuh"
 #include "sr_route_math.cuh"
+#include "sr_timeline.cuh"
 
 #ifndef SR_DECODE_RB
 #define SR_DECODE_RB 1 // row blocks of 16 per consumer warp and tile
@@ -54,6 +55,8 @@
 #ifndef SR_DECODE_STAGES
 #define SR_DECODE_STAGES 4
 #endif
+
+SR_TL_DEFINE(tl_decode)
 
 namespace sr {
 namespace {
@@ -66,8 +69,9 @@ constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeThreads = 32 * kCWarps;
-constexpr int kCosBuf = kCWarps * kMaxGroup * kHeadDim; // floats of the comb scratch, reused by fused routing
 constexpr int kMergeBatch = 16; // partials in flight per thread in the final merge
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kFastUnits = 32; // launches with at most this many units plan in registers
 
 struct alignas(16) TileHdr {
     int32_t unit;       // flat unit b*Hkv+g
@@ -80,7 +84,10 @@ struct alignas(16) TileHdr {
     int32_t pad;
 };
 
-constexpr int kSeqTab = 4096; // seq_lens entries staged in shared memory
+#ifndef SR_DECODE_SEQTAB
+#define SR_DECODE_SEQTAB 4096
+#endif
+constexpr int kSeqTab = SR_DECODE_SEQTAB; // seq_lens entries staged in shared memory
 
 struct Misc {
     int abort_flag;
@@ -91,6 +98,7 @@ struct Misc {
     long long wsum[kCWarps + 1];
     int first_bad; // first malformed entry of the active list (INT_MAX: none)
     int first_u;   // unit of the producer's first active entry (-1: none)
+    uint8_t sflag[32]; // fused routing of at most 32 units: sink flags
 };
 
 struct Params {
@@ -216,54 +224,36 @@ __device__ __forceinline__ long long block_scan(long long x, Misc *misc, long lo
     return before + v;
 }
 
-// Fused routing: sflag[u] = sink for every unit, read straight from global
-// memory, one half-warp per (unit, head) pair. Every CTA computes the same
-// decisions as the routing kernel (the same arithmetic, sr_route_math.cuh);
-// CTA 0 also writes the route mask.
+// Fused routing: every CTA routes every unit itself with the routing kernel's
+// arithmetic (sr_route_math.cuh, one warp per GQA group, loads straight from
+// global memory), so its decisions equal sr_route's bit for bit; CTA 0 also
+// writes the route mask. flag[u] = sink. Called by all threads; no barrier.
 template <int M>
-__device__ __forceinline__ void route_units(const Params &p, int U, uint8_t *sflag, float *cosbuf)
+__device__ __forceinline__ void route_all_units(const Params &p, int U, uint8_t *flag)
 {
-    // Units in chunks whose cosines fit cosbuf (kCosBuf floats); per round each
-    // half-warp loads the blocks of 4 pairs before reducing any of them.
-    constexpr int kChunkUnits = kCosBuf / M;
-    constexpr int kHalfWarps = kThreads / 16;
-    const int hw = (int)threadIdx.x >> 4, l16 = (int)threadIdx.x & 15;
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int u0 = 0; u0 < U; u0 += kChunkUnits) {
-        const int nu = (U - u0) < kChunkUnits ? (U - u0) : kChunkUnits;
-        const int pairs = nu * M;
-        for (int base = 0; base < pairs; base += 4 * kHalfWarps) {
-            uint4 qv[4], kv[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int pr = base + r * kHalfWarps + hw;
-                const bool valid = pr < pairs;
-                // q row (u0*M + pr) of [B*Hq, 128]; k0 row of unit u0 + pr/M
-                qv[r] = valid ? __ldg(reinterpret_cast<const uint4 *>(p.q + ((size_t)u0 * M + pr) * kHeadDim) + l16)
-                              : zero;
-                kv[r] = valid ? __ldg(reinterpret_cast<const uint4 *>(p.k0 + ((size_t)u0 + pr / M) * kHeadDim) + l16)
-                              : zero;
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int pr = base + r * kHalfWarps + hw;
-                const float c = pair_cosine(qv[r], kv[r]);
-                if (pr < pairs && l16 == 0)
-                    cosbuf[pr] = c;
-            }
-        }
-        __syncthreads();
-        for (int lu = (int)threadIdx.x; lu < nu; lu += kThreads) {
-            float s = INFINITY;
-#pragma unroll
-            for (int m = 0; m < M; ++m)
-                s = fminf(s, cosbuf[lu * M + m]);
-            const uint8_t sink = (s >= p.tau) ? 1 : 0;
-            sflag[u0 + lu] = sink;
-            if (blockIdx.x == 0 && p.mask_out)
-                p.mask_out[u0 + lu] = sink;
-        }
-        __syncthreads();
+    route_units_warp<M, true>(reinterpret_cast<const uint4 *>(p.q), reinterpret_cast<const uint4 *>(p.k0), U, p.tau,
+                              (int)threadIdx.x >> 5, kThreads / 32, [&](int u, bool sink) {
+                                  flag[u] = sink ? 1 : 0;
+                                  if (blockIdx.x == 0 && p.mask_out)
+                                      p.mask_out[u] = sink ? 1 : 0;
+                              });
+}
+
+__device__ __forceinline__ void route_all_units(const Params &p, int U, uint8_t *flag, int M)
+{
+    switch (M) {
+    case 1:
+        route_all_units<1>(p, U, flag);
+        break;
+    case 2:
+        route_all_units<2>(p, U, flag);
+        break;
+    case 4:
+        route_all_units<4>(p, U, flag);
+        break;
+    default:
+        route_all_units<8>(p, U, flag);
+        break;
     }
 }
 
@@ -290,6 +280,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const uint32_t cbar = smem_u32(&bars[2 * STAGES]);
 
     // ---------------------------------------------------------------- prologue
+    if (tid == 0)
+        SR_STAMP(tl_decode, 0);
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
@@ -312,7 +304,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         bitmap[w] = 0;
     __syncthreads();
     // Prologue tables in the stage buffers (free until the first copy),
-    // sized by the actual batch and unit count.
+    // sized by the actual batch and unit count (launches with more than
+    // kFastUnits units only).
     const bool seq_smem = p.B <= kSeqTab;
     int32_t *seqtab = reinterpret_cast<int32_t *>(smem + C::OFF_SEQ);
     int32_t *ltab = reinterpret_cast<int32_t *>(smem);
@@ -320,14 +313,89 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     uint8_t *sflag = smem + ((4 * U + 127) & ~127) + ((2 * U + 127) & ~127);
     int errbits = 0;
     int n = 0;
+    long long P = 0;
+    // Launches with at most 32 units: every warp derives the active set in
+    // registers from one round of loads (lane r holds the active entry of rank
+    // r, its length and the inclusive prefix of the lengths), so no block
+    // barrier follows the dependency wait. The producer warp finds its share
+    // with a ballot and issues its first copies at once; the consumer warps do
+    // the sink bypass from their own copy of the set.
+    const bool fast = U <= kFastUnits;
+    uint32_t act_bits = 0;
+    int lane_unit = 0, lane_len = 0;
+    long long lane_incl = 0;
     long long local = 0;
-    if constexpr (!FUSED) {
+    if (fast) {
+        grid_dependency_wait();
+        grid_launch_dependents();
+        if (tid == 0)
+            SR_STAMP(tl_decode, 1);
+        // All inputs are read after the wait: the preceding kernel may write
+        // any of them (the routing kernel the list, the append step seq_lens).
+        const int sl = (lane < p.B) ? __ldg(p.seq_lens + lane) : 1;
+        if constexpr (!FUSED) {
+            n = __ldg(p.active);
+            const int e = (lane < U) ? __ldg(p.active + 1 + lane) : -1;
+            if (n < 0 || n > U) {
+                errbits |= SR_DEVERR_ACTIVE_LIST;
+                n = n < 0 ? 0 : U;
+            }
+            // Keep the longest well-formed prefix (entries in range and
+            // strictly ascending); a malformed entry ends it and is reported.
+            const int prev = __shfl_up_sync(kFull, e, 1);
+            const unsigned bad = __ballot_sync(kFull, lane < n && (e < 0 || e >= U || (lane > 0 && e <= prev)));
+            if (bad) {
+                errbits |= SR_DEVERR_ACTIVE_LIST;
+                n = __ffs(bad) - 1;
+            }
+            lane_unit = (lane < n) ? e : 0;
+            act_bits = __reduce_or_sync(kFull, (lane < n) ? (1u << lane_unit) : 0u);
+        } else {
+            route_all_units(p, U, misc->sflag, M);
+            __syncthreads();
+            act_bits = __ballot_sync(kFull, lane < U && !misc->sflag[lane]);
+            n = __popc(act_bits);
+            const int r = (int)__fns(act_bits, 0, lane + 1); // unit of rank `lane`
+            lane_unit = (lane < n && r >= 0 && r < U) ? r : 0;
+            if (blockIdx.x == 0 && warp == kCWarps && p.active_out) {
+                if (lane < n)
+                    p.active_out[1 + lane] = lane_unit;
+                if (lane == 0)
+                    p.active_out[0] = n;
+            }
+        }
+        int L = __shfl_sync(kFull, sl, lane_unit / p.Hkv);
+        if (__ballot_sync(kFull, lane < n && (L < 1 || L > p.Lmax)))
+            errbits |= SR_DEVERR_SEQ_LEN;
+        L = L < 1 ? 1 : (L > p.Lmax ? p.Lmax : L);
+        lane_len = (lane < n) ? L : 0;
+        lane_incl = lane_len;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(kFull, lane_incl, o);
+            if (lane >= o)
+                lane_incl += y;
+        }
+        P = __shfl_sync(kFull, lane_incl, 31);
+        if (warp == kCWarps) { // the tables the producer lane walks
+            if (lane < p.B)
+                seqtab[lane] = sl;
+            if (lane == 0)
+                bitmap[0] = act_bits;
+        }
+        if (tid == 0)
+            SR_STAMP(tl_decode, 2);
+        if (errbits && blockIdx.x == 0 && warp == kCWarps && lane == 0)
+            atomicOr(p.err, errbits);
+    } else if constexpr (!FUSED) {
         // The preceding kernel may have written every input (the routing
         // kernel writes the active list; the append step also advances
         // seq_lens), so all of them are read after the dependency wait, the
         // length table and the list count in the same round trip.
         grid_dependency_wait();
         grid_launch_dependents();
+        if (tid == 0)
+            SR_STAMP(tl_decode, 1);
         __syncthreads();
 
         n = __ldg(p.active);
@@ -351,6 +419,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 utab[i] = (int16_t)u;
         }
         __syncthreads();
+        if (tid == 0)
+            SR_STAMP(tl_decode, 2);
         if (misc->first_bad < n) {
             errbits |= SR_DEVERR_ACTIVE_LIST;
             n = misc->first_bad;
@@ -374,23 +444,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         if (seq_smem)
             for (int b = tid; b < p.B; b += kThreads)
                 seqtab[b] = __ldg(p.seq_lens + b);
-        // One thread per (unit, head) pair reads both rows straight from
-        // global memory. (Staging them with bulk copies in every CTA was
-        // measured slower: 148 CTAs copying the same few KB serialise.)
-        switch (M) {
-        case 1:
-            route_units<1>(p, U, sflag, comb);
-            break;
-        case 2:
-            route_units<2>(p, U, sflag, comb);
-            break;
-        case 4:
-            route_units<4>(p, U, sflag, comb);
-            break;
-        default:
-            route_units<8>(p, U, sflag, comb);
-            break;
-        }
+        route_all_units(p, U, sflag, M);
         __syncthreads();
         // Ordered compaction of the active units into the same tables the
         // work-list path builds.
@@ -418,10 +472,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         if (blockIdx.x == 0 && tid == 0 && p.active_out)
             p.active_out[0] = n;
     }
-    long long P;
-    (void)block_scan(local, misc, &P);
-    if (errbits && blockIdx.x == 0)
-        atomicOr(p.err, errbits);
+    if (!fast) {
+        (void)block_scan(local, misc, &P);
+        if (errbits && blockIdx.x == 0)
+            atomicOr(p.err, errbits);
+    }
 
     const int G = gridDim.x;
     long long chunk = 1, r0 = 0, r1 = 0;
@@ -431,7 +486,32 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         chunk = chunk < kMinChunk ? kMinChunk : chunk;
         r0 = (long long)blockIdx.x * chunk;
         r1 = r0 + chunk < P ? r0 + chunk : P;
-        if (r0 < P) { // find the active entry whose positions contain r0
+    }
+    if (fast) {
+        if (warp == kCWarps) {
+            // This CTA's first active entry: the rank whose positions contain
+            // r0 (automatic splits), or rank 0 (forced splits).
+            int i0 = INT_MAX;
+            long long s0 = 0;
+            if (p.n_splits != 0) {
+                i0 = 0;
+            } else if (P > 0 && r0 < P) {
+                // never empty: the last valid lane holds the total P > r0
+                const unsigned gt = __ballot_sync(kFull, lane < n && lane_incl > r0);
+                const int i = gt ? __ffs(gt) - 1 : 0;
+                s0 = __shfl_sync(kFull, lane_incl - lane_len, i);
+                i0 = gt ? i : INT_MAX;
+            }
+            const int fu = (i0 < n) ? __shfl_sync(kFull, lane_unit, i0 < 32 ? i0 : 0) : -1;
+            if (lane == 0) {
+                misc->i0 = i0;
+                misc->s0 = s0;
+                misc->first_u = fu;
+            }
+            __syncwarp();
+        }
+    } else {
+        if (p.n_splits == 0 && P > 0 && r0 < P) { // find the active entry whose positions contain r0
             long long carry = 0;
             for (int base = 0; base < n; base += kThreads) {
                 const int i = base + tid;
@@ -446,19 +526,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 carry += tot;
             }
         }
+        // Generic stores into the stage buffers (tables) must be ordered
+        // before the TMA writes that will reuse those bytes.
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            // The producer walks the active units in the bitmap from its first
+            // entry on (rank i0 for automatic splits, rank 0 for forced ones).
+            const int i0 = (p.n_splits == 0) ? misc->i0 : 0;
+            misc->i0 = i0;
+            misc->first_u = (i0 < n) ? (int)utab[i0] : -1;
+        }
+        __syncthreads(); // the stage buffers are free for the copies from here on
     }
-    // Generic stores into the stage buffers (tables) must be ordered before
-    // the TMA writes that will reuse those bytes.
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        // The producer walks the active units in the bitmap from its first
-        // entry on (rank i0 for automatic splits, rank 0 for forced ones).
-        const int i0 = (p.n_splits == 0) ? misc->i0 : 0;
-        misc->i0 = i0;
-        misc->first_u = (i0 < n) ? (int)utab[i0] : -1;
-    }
-    __syncthreads(); // the stage buffers are free for the copies from here on
+    if (fast ? tid == 32 * kCWarps : tid == 0)
+        SR_STAMP(tl_decode, 3);
 
     // ---------------------------------------------------------------- producer
     if (warp == kCWarps) {
@@ -490,6 +572,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 }
                 if (qbytes)
                     bulk_load(smem_u32(smem + C::OFF_Q + stage * C::QBYTES), qsrc, qbytes, fb);
+                if (issued_parity[stage] < 0 && stage == 0 && ph == 0)
+                    SR_STAMP(tl_decode, 4);
                 issued_parity[stage] = (int)ph;
             } else {
                 mbar_arrive(fb);
@@ -568,6 +652,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             h.unit = -1;
             h.flags = kEnd;
             ok = emit(h, nullptr, 0);
+            SR_STAMP(tl_decode, 14);
         }
         if (!ok) {
             atomicOr(p.err, SR_DEVERR_TIMEOUT);
@@ -590,7 +675,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     {
         const int gw = blockIdx.x * kCWarps + w, nw = gridDim.x * kCWarps;
         for (int u = gw; u < U; u += nw) {
-            if (bitmap[u >> 5] & (1u << (u & 31)))
+            if (fast ? ((act_bits >> u) & 1u) : (bitmap[u >> 5] & (1u << (u & 31))))
                 continue;
             const int b = u / p.Hkv, gg = u - b * p.Hkv;
             const size_t row0 = (size_t)b * p.Hq + (size_t)gg * M;
@@ -613,6 +698,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         }
     }
 
+    if (ctid == 0)
+        SR_STAMP(tl_decode, 5);
     const uint32_t sbase = smem_u32(smem);
     uint32_t rowK[RB], rowV[RB];
 #pragma unroll
@@ -662,11 +749,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         return __all_sync(0xffffffffu, r);
     };
 
+#ifdef SR_TIMELINE
+    bool tl_first = true;
+    int tl_splits = 0, tl_last = 0;
+#endif
     for (;;) {
         if (!__all_sync(0xffffffffu, wait_bar(full0 + 8 * stage, ph, abort_flag))) {
             ok = false;
             break;
         }
+#ifdef SR_TIMELINE
+        if (tl_first && ctid == 0)
+            SR_STAMP(tl_decode, 6);
+        tl_first = false;
+#endif
         const TileHdr h = hdr[stage];
         if (h.flags & kEnd)
             break;
@@ -788,6 +884,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             mbar_arrive(empty0 + 8 * stage);
 
         if (h.flags & kLast) {
+#ifdef SR_TIMELINE
+            if (ctid == 0)
+                SR_STAMP(tl_decode, 7);
+            ++tl_splits;
+#endif
             // ---- merge the four warps' states into one partial of this split
             float l0 = lrun[0], l1 = lrun[1];
 #pragma unroll
@@ -799,58 +900,51 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 mlsm[w * kMaxGroup + 2 * t] = make_float2(mrun[0], l0);
                 mlsm[w * kMaxGroup + 2 * t + 1] = make_float2(mrun[1], l1);
             }
-            if (!(ok = cbar_sync()))
-                break;
-            float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-            for (int ww = 0; ww < kCWarps; ++ww) {
-                M0 = fmaxf(M0, mlsm[ww * kMaxGroup + 2 * t].x);
-                M1 = fmaxf(M1, mlsm[ww * kMaxGroup + 2 * t + 1].x);
-            }
-            const float f0 = (M0 == -INFINITY) ? 0.f : exp2f(mrun[0] - M0);
-            const float f1 = (M1 == -INFINITY) ? 0.f : exp2f(mrun[1] - M1);
+            // Unscaled O of this warp; the readers below weight the four warps.
             float *cw = comb + w * (kMaxGroup * kHeadDim);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int d0 = 16 * j + g;
                 if (2 * t < M) {
-                    cw[(2 * t) * kHeadDim + d0] = o[j][0] * f0;
-                    cw[(2 * t) * kHeadDim + d0 + 8] = o[j][2] * f0;
+                    cw[(2 * t) * kHeadDim + d0] = o[j][0];
+                    cw[(2 * t) * kHeadDim + d0 + 8] = o[j][2];
                 }
                 if (2 * t + 1 < M) {
-                    cw[(2 * t + 1) * kHeadDim + d0] = o[j][1] * f1;
-                    cw[(2 * t + 1) * kHeadDim + d0 + 8] = o[j][3] * f1;
+                    cw[(2 * t + 1) * kHeadDim + d0] = o[j][1];
+                    cw[(2 * t + 1) * kHeadDim + d0 + 8] = o[j][3];
                 }
             }
             if (!(ok = cbar_sync()))
                 break;
+            // Partial of the split, one float4 column per thread: the warps'
+            // states weighted by 2^(m_w - max_w m_w) (0 for a warp that saw no
+            // row of this split).
             float *po = p.part_o + (size_t)h.slot * M * kHeadDim;
             for (int idx = ctid; idx < M * 32; idx += 32 * kCWarps) {
                 const int head = idx >> 5, d4 = (idx & 31) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int ww = 0; ww < kCWarps; ++ww) {
-                    const float4 x =
-                        *reinterpret_cast<const float4 *>(comb + ww * (kMaxGroup * kHeadDim) + head * kHeadDim + d4);
-                    acc.x += x.x, acc.y += x.y, acc.z += x.z, acc.w += x.w;
-                }
-                __stcg(reinterpret_cast<float4 *>(po + head * kHeadDim + d4), acc);
-            }
-            if (ctid < M) {
+                float2 ml[kCWarps];
                 float Mh = -INFINITY;
 #pragma unroll
-                for (int ww = 0; ww < kCWarps; ++ww)
-                    Mh = fmaxf(Mh, mlsm[ww * kMaxGroup + ctid].x);
-                float Lh = 0.f;
-                if (Mh != -INFINITY) {
-#pragma unroll
-                    for (int ww = 0; ww < kCWarps; ++ww) {
-                        const float2 x = mlsm[ww * kMaxGroup + ctid];
-                        if (x.x != -INFINITY)
-                            Lh += x.y * exp2f(x.x - Mh);
-                    }
+                for (int ww = 0; ww < kCWarps; ++ww) {
+                    ml[ww] = mlsm[ww * kMaxGroup + head];
+                    Mh = fmaxf(Mh, ml[ww].x);
                 }
-                __stcg(p.part_ml + (size_t)h.slot * M + ctid, make_float2(Mh, Lh));
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                float Lh = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < kCWarps; ++ww) {
+                    const float f = (ml[ww].x == -INFINITY) ? 0.f : exp2f(ml[ww].x - Mh);
+                    const float4 x =
+                        *reinterpret_cast<const float4 *>(comb + ww * (kMaxGroup * kHeadDim) + head * kHeadDim + d4);
+                    acc.x = fmaf(x.x, f, acc.x);
+                    acc.y = fmaf(x.y, f, acc.y);
+                    acc.z = fmaf(x.z, f, acc.z);
+                    acc.w = fmaf(x.w, f, acc.w);
+                    Lh = fmaf(ml[ww].y, f, Lh);
+                }
+                __stcg(reinterpret_cast<float4 *>(po + head * kHeadDim + d4), acc);
+                if (d4 == 0)
+                    __stcg(p.part_ml + (size_t)h.slot * M + head, make_float2(Mh, Lh));
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -865,9 +959,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             if (!(ok = cbar_sync()))
                 break;
             if (ctid == 0)
+                SR_STAMP(tl_decode, 8);
+            if (ctid == 0)
                 misc->is_last = (atom_add_acq_rel_gpu(p.cnt + h.unit, 1) == h.nseg - 1) ? 1 : 0;
             if (!(ok = cbar_sync()))
                 break;
+            if (ctid == 0)
+                SR_STAMP(tl_decode, 9);
             if (misc->is_last) {
                 // ---- last split of the unit to finish: merge all its partials.
                 // Threads own float4 columns of the unit's [M x 128] output;
@@ -961,6 +1059,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 // Shared scratch (comb, mlsm) is reused by the next split's end.
                 if (!(ok = cbar_sync()))
                     break;
+#ifdef SR_TIMELINE
+                if (ctid == 0)
+                    SR_STAMP(tl_decode, 10);
+                ++tl_last;
+#endif
             }
         }
         if (++stage == STAGES) {
@@ -970,6 +1073,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     }
     if (!ok && lane == 0)
         atomicOr(p.err, SR_DEVERR_TIMEOUT);
+#ifdef SR_TIMELINE
+    if (ctid == 0) {
+        SR_STAMP(tl_decode, 11);
+        tl_decode[blockIdx.x][12] = (unsigned long long)tl_splits;
+        tl_decode[blockIdx.x][13] = (unsigned long long)tl_last;
+    }
+#endif
 }
 
 // ---- host side ------------------------------------------------------------------------

@@ -27,7 +27,7 @@
 // slot, and stage the group's position-0 key (the captured one at slot 0, else
 // the stored k0); eight threads per query row rotate it into q_out and the
 // staged rows; the staged rows are routed with the routing kernel's own
-// routine (one half-warp per pair), so the decision equals sr_route on
+// routine (one warp per GQA group), so the decision equals sr_route on
 // (q_out, k0) bit for bit. Lengths advance after every read of
 // them; the compaction is the routing kernel's.
 #include <atomic>
@@ -124,7 +124,6 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
     extern __shared__ __align__(128) uint8_t dsm[]; // [cu*(M+1)*256 staged rows][B*Hkv sink flags]
     __shared__ int32_t warp_cnt[kWarps];
     __shared__ int32_t warp_off[kWarps + 1];
-    __shared__ float cosbuf[chunk_units<M>() * M];
 
     const int U = p.B * p.Hkv;
     uint4 *rows = reinterpret_cast<uint4 *>(dsm);
@@ -211,7 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
             qd[j + 8] = hi;
         }
         __syncthreads();
-        route_staged<M, kThreads>(rows, u0, nu, p.tau, sink_flag, p.mask, cosbuf);
+        route_units_warp<M, false>(rows, krows, nu, p.tau, (int)threadIdx.x >> 5, kWarps, [&](int lu, bool sink) {
+            sink_flag[u0 + lu] = sink ? 1 : 0;
+            p.mask[u0 + lu] = sink ? 1 : 0;
+        });
         __syncthreads(); // the rows are overwritten by the next chunk
     }
 

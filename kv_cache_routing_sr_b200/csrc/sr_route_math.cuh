@@ -1,7 +1,7 @@
-// Cosine of one query head with its group's position-0 key and the ordered
-// compaction of the active units, shared by the routing kernel, the fused
-// route + decode prologue and the RoPE + append + route step, so that all of
-// them take the same decision bit for bit.
+// Cosine of one query head with its group's position-0 key, the minimum over
+// the group's heads, and the ordered compaction of the active units, shared by
+// the routing kernel, the fused route + decode prologue and the RoPE + append
+// + route step, so that all of them take the same decision bit for bit.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -9,17 +9,25 @@
 
 namespace sr {
 
-// The cosine of a (unit, head) pair is computed by the 16 lanes of a
-// half-warp: lane l takes the 16-byte block l (elements 8l .. 8l+7) of the
-// query row and of the key row, sums its 8 products in element order, and a
-// fixed xor-shuffle tree (offsets 8, 4, 2, 1) adds the 16 lane sums. Every
-// caller uses this one arithmetic, so they all take the same decision bit for
-// bit.
+// Lane mapping of the routing arithmetic for group size M: W lanes take one
+// (unit, query head) pair, each lane V consecutive 16-byte blocks (8V bf16
+// elements) of the query row and of the group's key row. A warp holds 32 / W
+// pairs: exactly one GQA group when M >= 4 (one warp per group), 4 / M groups
+// when M < 4. Every caller (routing kernel, fused route + decode prologue,
+// RoPE + append + route step) uses this one arithmetic, so they all take the
+// same decision bit for bit.
+template <int M> struct RouteLanes {
+    static_assert(M == 1 || M == 2 || M == 4 || M == 8, "group size");
+    static constexpr int W = (M == 8) ? 4 : 8; // lanes per pair
+    static constexpr int V = 16 / W;           // 16-byte blocks of each row per lane
+    static constexpr int PAIRS = 32 / W;       // pairs per warp
+    static constexpr int UNITS = PAIRS / M;    // units per warp
+};
 
-// Lane sums of <a,b>, <a,a> and <b,b> over one 16-byte block (8 bf16) of each row.
-__device__ __forceinline__ void dots_vec(const uint4 &a, const uint4 &b, float &ab, float &aa, float &bb)
+// Adds the products of one 16-byte block (8 bf16) of a and b to ab, aa, bb,
+// in element order.
+__device__ __forceinline__ void dots_block(const uint4 &a, const uint4 &b, float &ab, float &aa, float &bb)
 {
-    ab = aa = bb = 0.f;
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
     const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -35,75 +43,94 @@ __device__ __forceinline__ void dots_vec(const uint4 &a, const uint4 &b, float &
     }
 }
 
-// Sum over the 16 lanes of each half-warp; every lane receives it. All 32
-// lanes of the warp must call it.
-__device__ __forceinline__ float half_warp_sum(float x)
+// s_g = min over the group's heads of cos(q_h, k0_g), from this lane's blocks
+// (qv of its query row, kv of its key row). The W lanes of a pair add their
+// sums with a fixed xor tree; the cosine is 0 when a norm is 0, and a NaN
+// cosine counts as +inf so that it never lowers the minimum; an xor tree over
+// the group's lanes takes the minimum. Every lane of the group receives s_g.
+// All 32 lanes must call it.
+template <int M>
+__device__ __forceinline__ float group_min_cosine(const uint4 (&qv)[RouteLanes<M>::V],
+                                                  const uint4 (&kv)[RouteLanes<M>::V])
 {
+    constexpr int W = RouteLanes<M>::W, V = RouteLanes<M>::V;
+    float ab = 0.f, aa = 0.f, bb = 0.f;
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1)
-        x += __shfl_xor_sync(0xffffffffu, x, off);
-    return x;
-}
-
-// cos(q_h, k0_g) of one pair from this lane's blocks: 0 when a norm is 0; a
-// NaN result is returned as +inf so that it never lowers the group minimum.
-// Returned in all 16 lanes of the half-warp. All 32 lanes must call it.
-__device__ __forceinline__ float pair_cosine(const uint4 &qv, const uint4 &kv)
-{
-    float ab, aa, bb;
-    dots_vec(qv, kv, ab, aa, bb);
-    ab = half_warp_sum(ab);
-    aa = half_warp_sum(aa);
-    bb = half_warp_sum(bb);
+    for (int v = 0; v < V; ++v)
+        dots_block(qv[v], kv[v], ab, aa, bb);
+#pragma unroll
+    for (int off = W / 2; off > 0; off >>= 1) {
+        ab += __shfl_xor_sync(0xffffffffu, ab, off);
+        aa += __shfl_xor_sync(0xffffffffu, aa, off);
+        bb += __shfl_xor_sync(0xffffffffu, bb, off);
+    }
     float c = (aa == 0.f || bb == 0.f) ? 0.f : ab / (sqrtf(aa) * sqrtf(bb));
     if (c != c)
         c = INFINITY;
+#pragma unroll
+    for (int off = W; off < W * M; off <<= 1)
+        c = fminf(c, __shfl_xor_sync(0xffffffffu, c, off));
     return c;
 }
 
-// Route the nu units u0 .. u0+nu-1 whose rows are staged in shared memory:
-// `rows` holds their nu*M query rows (row u*M+m of q) followed by their nu key
-// rows, 256 bytes each. NT threads (a multiple of 32) take NT/8 pairs per
-// pass, two per half-warp; the pairs' cosines go to cosbuf (nu*M floats), and
-// after a block barrier one thread per unit takes the minimum over its M heads.
-// Writes sflag[u] = sink, and mask_out[u] when mask_out is not null. Called by
-// all NT threads; ends without a trailing barrier.
-template <int M, int NT>
-__device__ __forceinline__ void route_staged(const uint4 *rows, int u0, int nu, float tau, uint8_t *sflag,
-                                             uint8_t *mask_out, float *cosbuf)
+// This lane's blocks of warp chunk `chunk` (units chunk*UNITS ..): qrows holds
+// nu*M query rows (row u*M+m) and krows nu key rows, 16 blocks each, in global
+// memory (kGlobal: read-only loads) or shared memory. Units past nu read as
+// zero. Returns this lane's unit.
+template <int M, bool kGlobal>
+__device__ __forceinline__ int load_route_blocks(const uint4 *qrows, const uint4 *krows, int nu, int chunk,
+                                                 uint4 (&qv)[RouteLanes<M>::V], uint4 (&kv)[RouteLanes<M>::V])
 {
-    const uint4 *kr = rows + nu * M * 16;
-    const int pairs = nu * M;
-    const int hw = (int)threadIdx.x >> 4, l16 = (int)threadIdx.x & 15;
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    // Two pairs per half-warp and pass: their loads and shuffle chains are
-    // independent, so they overlap (each pair's arithmetic is unchanged).
-    for (int base = 0; base < pairs; base += NT / 8) {
-        const int pa = base + hw, pb = base + NT / 16 + hw;
-        const bool va = pa < pairs, vb = pb < pairs;
-        const uint4 qa = va ? rows[pa * 16 + l16] : zero;
-        const uint4 ka = va ? kr[(pa / M) * 16 + l16] : zero;
-        const uint4 qb = vb ? rows[pb * 16 + l16] : zero;
-        const uint4 kb = vb ? kr[(pb / M) * 16 + l16] : zero;
-        const float ca = pair_cosine(qa, ka);
-        const float cb = pair_cosine(qb, kb);
-        if (l16 == 0) {
-            if (va)
-                cosbuf[pa] = ca;
-            if (vb)
-                cosbuf[pb] = cb;
+    using RL = RouteLanes<M>;
+    const int lane = (int)threadIdx.x & 31;
+    const int pr = lane / RL::W, j = lane % RL::W;
+    const int unit = chunk * RL::UNITS + pr / M;
+    const size_t qrow = (size_t)chunk * RL::PAIRS + pr;
+#pragma unroll
+    for (int v = 0; v < RL::V; ++v) {
+        if (unit < nu) {
+            const uint4 *qp = qrows + qrow * 16 + j * RL::V + v;
+            const uint4 *kp = krows + (size_t)unit * 16 + j * RL::V + v;
+            qv[v] = kGlobal ? __ldg(qp) : *qp;
+            kv[v] = kGlobal ? __ldg(kp) : *kp;
+        } else {
+            qv[v] = make_uint4(0u, 0u, 0u, 0u);
+            kv[v] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
-    __syncthreads();
-    for (int lu = (int)threadIdx.x; lu < nu; lu += NT) {
-        float s = INFINITY;
+    return unit;
+}
+
+// Routes units 0 .. nu-1: warp `wid` of `nwarps` takes the warp chunks wid,
+// wid + nwarps, ..., and issues the loads of its next chunk before reducing
+// the current one. For every unit one lane calls store(u, sink), sink being
+// (s_g >= tau). Called by whole warps; no block barrier inside.
+template <int M, bool kGlobal, typename Store>
+__device__ __forceinline__ void route_units_warp(const uint4 *qrows, const uint4 *krows, int nu, float tau, int wid,
+                                                 int nwarps, Store &&store)
+{
+    using RL = RouteLanes<M>;
+    const int lane = (int)threadIdx.x & 31;
+    const int nchunks = (nu + RL::UNITS - 1) / RL::UNITS;
+    int c = wid;
+    if (c >= nchunks)
+        return;
+    uint4 qa[RL::V], ka[RL::V];
+    int ua = load_route_blocks<M, kGlobal>(qrows, krows, nu, c, qa, ka);
+    for (; c < nchunks; c += nwarps) {
+        uint4 qb[RL::V], kb[RL::V];
+        int ub = nu;
+        if (c + nwarps < nchunks)
+            ub = load_route_blocks<M, kGlobal>(qrows, krows, nu, c + nwarps, qb, kb);
+        const float s = group_min_cosine<M>(qa, ka);
+        if (lane % (RL::W * M) == 0 && ua < nu)
+            store(ua, s >= tau);
 #pragma unroll
-        for (int m = 0; m < M; ++m)
-            s = fminf(s, cosbuf[lu * M + m]);
-        const uint8_t sink = (s >= tau) ? 1 : 0;
-        sflag[u0 + lu] = sink;
-        if (mask_out)
-            mask_out[u0 + lu] = sink;
+        for (int v = 0; v < RL::V; ++v) {
+            qa[v] = qb[v];
+            ka[v] = kb[v];
+        }
+        ua = ub;
     }
 }
 

@@ -4,7 +4,6 @@
 // this library instead of a caller-provided workspace. Nothing here allocates:
 // no cudaMalloc / cudaFree, no library allocator.
 #include <cuda_runtime.h>
-#include <mutex>
 
 #include "sinkrouter.h"
 #include "sr_internal.h"
@@ -13,35 +12,22 @@ namespace {
 
 // One array per GPU that loads the library, kept until the process exits.
 // In host code this name is only a stand-in for the symbol: its device address
-// comes from cudaGetSymbolAddress (once per device, below).
+// comes from cudaGetSymbolAddress (below, with the caller's device current).
 static __device__ __align__(256) unsigned char g_static_scratch[SR_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices];
-std::mutex g_scratch_mu;
-
-// Device address of g_static_scratch on the current device. The first call on
-// a device looks it up (this may load the module on that device); later calls
-// reuse it.
+// Device address of g_static_scratch on the current device, looked up on
+// every call (cheap once the module is loaded on that device), so that no
+// address outlives a device reset. The first call on a device may load the
+// module there.
 cudaError_t scratch_address(void **addr)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess)
-            return e;
-        if (!p)
-            return cudaErrorInvalidSymbol;
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    if (!p)
+        return cudaErrorInvalidSymbol;
+    *addr = p;
     return cudaSuccess;
 }
 

@@ -46,13 +46,17 @@ EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_dec
            "sr_combine_partials", "sr_selftest_bounded_wait"]
 
 
-def load(path: str = LIBRARY):
-    """Load (once) and type the library. The in-tree library is compiled first
-    if it is absent (nvcc, sm_100a); any other missing path, or a failed
-    compile, raises: there is no other implementation to fall back to."""
+def load(path: str | None = None):
+    """Load (once) and type the library: `path`, else the file named by the
+    SINKROUTER_LIBRARY environment variable (another build of the same
+    sources), else the in-tree library, which is compiled first if it is
+    absent (nvcc, sm_100a). Any other missing path, or a failed compile,
+    raises: there is no other implementation to fall back to."""
     global _lib
     if _lib is not None:
         return _lib
+    if path is None:
+        path = os.environ.get("SINKROUTER_LIBRARY") or LIBRARY
     if not os.path.exists(path) and os.path.abspath(path) == os.path.abspath(LIBRARY):
         from . import build as _build
         try:

@@ -5,6 +5,7 @@ import pytest
 import torch
 
 import math
+import os
 
 import oracle
 from kv_cache_routing_sr_b200 import inputs, native, proxy_quality
@@ -127,14 +128,12 @@ def test_decode_full_size_sampled(name):
     H.check_against_oracle(x, out_g, mask_g, units=_sample(mask_g), what=name)
 
 
-@pytest.mark.parametrize("name", ["llama8b_128k", "llama70b_ragged", "llava7b_mha"])
-def test_decode_full_size_every_unit(name):
-    """Every unit of the full-size workload against the oracle (run once on the
-    whole problem, 8 threads): sink heads bit-exact v0, active heads within
-    the tolerances, per (sequence, head)."""
-    x = inputs.make(name, seed=21, device=DEV)
+def _every_unit(x, what):
+    """Every unit of a full-size workload against the oracle (run once on the
+    whole problem, one thread per host core): sink heads bit-exact v0, active
+    heads within the tolerances, per (sequence, head)."""
     mask_g, act_g, out_g, _ = H.gpu_step(x)
-    ref = H.oracle_full(x, x.tau, n_threads=8)
+    ref = H.oracle_full(x, x.tau, n_threads=os.cpu_count() or 8)
     H.assert_route_equal(mask_g, act_g, ref.mask, ref.active_list)
     Hkv, M = x.n_kv_heads, x.n_q_heads // x.n_kv_heads
     v0 = x.v0.cpu()
@@ -145,9 +144,27 @@ def test_decode_full_size_every_unit(name):
             H.assert_sink_exact(out_g[b, g * M:(g + 1) * M], v0[b, g])
         else:
             act.append((b, g))
-    got = torch.stack([out_g[b, g * M:(g + 1) * M] for b, g in act])
-    want = torch.stack([ref.out[b, g * M:(g + 1) * M] for b, g in act])
-    H.assert_active_close(got, want, f"{name}, all {len(act)} active units")
+    if act:
+        got = torch.stack([out_g[b, g * M:(g + 1) * M] for b, g in act])
+        want = torch.stack([ref.out[b, g * M:(g + 1) * M] for b, g in act])
+        H.assert_active_close(got, want, f"{what}, all {len(act)} active units")
+    return len(act)
+
+
+@pytest.mark.parametrize("name", ["llama8b_128k", "llama70b_ragged", "llava7b_mha"])
+def test_decode_full_size_every_unit(name):
+    _every_unit(inputs.make(name, seed=21, device=DEV), name)
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.5])
+def test_512k_every_unit(frac):
+    """The full-size 512K workload (8 groups of 524288 positions; the automatic
+    plan gives each active group about 37 splits at half sinks and 18.5 with
+    none, each split thousands of positions long): every group against the
+    oracle."""
+    x = inputs.make("llama8b_512k", seed=23, device=DEV, sink_fraction=frac)
+    n_act = _every_unit(x, f"512k frac={frac}")
+    assert n_act == 8 - round(8 * frac)
 
 
 @pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
@@ -433,8 +450,10 @@ def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
     bits (lse included) must not depend on the rest of the launch: unit 0
     alone (every CTA holds at most one split, so the merging CTA has no
     further work) against unit 0 among many active units (more splits than
-    CTAs: CTA j's split j is never its last). ns = 70 at M = 4, 40 at M = 8
-    and 140 at M = 1 take several batches of the merge."""
+    CTAs: CTA j's split j is never its last), and the first sequence as a
+    launch of its own, whose 8 units take the prologue's register path.
+    ns = 70 at M = 4, 40 at M = 8 and 140 at M = 1 take several batches of the
+    merge."""
     G = native.grid_size()
     Hkv = 8
     B = max(1, -(-(G + ns) // (ns * Hkv)) + 1)  # B*Hkv*ns > G + ns
@@ -449,17 +468,23 @@ def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
     assert U * ns > G + ns and ns <= G
     del x
     runs = {}
-    for name, units in (("alone", [0]), ("among_many", list(range(U)))):
+    # "one_sequence": the first sequence alone (8 units: the prologue's register
+    # path); the other two runs have more than 32 units (its block-wide path).
+    for name, nb, units in (("alone", B, [0]), ("among_many", B, list(range(U))), ("one_sequence", 1, [0])):
         act = torch.tensor([len(units)] + units, dtype=torch.int32, device=DEV)
-        ws = native.Workspace(B, Hkv * M, Hkv, L, max_splits=ns, device=DEV)
-        lse = torch.empty((B, Hkv * M), dtype=torch.float32, device=DEV)
-        out = native.decode_attention(q, kc, vc, k0, v0, sl, act, n_splits=ns, workspace=ws, lse=lse)
+        ws = native.Workspace(nb, Hkv * M, Hkv, L, max_splits=ns, device=DEV)
+        lse = torch.empty((nb, Hkv * M), dtype=torch.float32, device=DEV)
+        out = native.decode_attention(q[:nb].contiguous(), kc[:nb].contiguous(), vc[:nb].contiguous(),
+                                      k0[:nb].contiguous(), v0[:nb].contiguous(), sl[:nb].contiguous(), act,
+                                      n_splits=ns, workspace=ws, lse=lse)
         torch.cuda.synchronize()
         assert ws.device_error() == 0
         runs[name] = (out[0, :M].cpu(), lse[0, :M].cpu())
-    a, b = runs["alone"], runs["among_many"]
-    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)), "unit 0 depends on the other units"
-    assert torch.equal(a[1].view(torch.int32), b[1].view(torch.int32)), "lse of unit 0 depends on the other units"
+    a = runs["alone"]
+    for other in ("among_many", "one_sequence"):
+        b = runs[other]
+        assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)), f"unit 0 differs ({other})"
+        assert torch.equal(a[1].view(torch.int32), b[1].view(torch.int32)), f"lse of unit 0 differs ({other})"
     # and both agree with the oracle
     ref, _ = oracle.decode(q[:1, :M].cpu(), kc[:1, :1].cpu(), vc[:1, :1].cpu(), v0[:1, :1].cpu(),
                            sl[:1].cpu(), torch.zeros(1, dtype=torch.uint8))
