@@ -72,6 +72,11 @@ def parse_args(argv=None):
                     help="instead of the contract line: per-token attention latency of a 32-layer stack, "
                          "CUDA-graph captured, at 128K/256K/512K context, routed vs routing disabled")
     ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--profile", metavar="WORKLOAD", default=None,
+                    help="instead of the contract line: run --warmup + --steps eager two-call steps of one workload "
+                         "(optionally at --max-ctx) and print a one-line summary; the command the ncu captures in "
+                         "profiles/ run")
+    ap.add_argument("--max-ctx", type=int, default=None, help="context of the --profile workload")
     ap.add_argument("--proxy-quality", action="store_true",
                     help="instead of the contract line: precision / recall / F1 of the cosine routing proxy "
                          "against the full-attention position-0 weight, on graded synthetic inputs")
@@ -149,8 +154,8 @@ def describe_config(x, n_active, n_gpus):
         "batch": x.batch, "context": x.max_seq_len, "q_heads": x.n_q_heads, "kv_heads": x.n_kv_heads,
         "head_dim": 128, "tau": x.tau, "units": x.batch * x.n_kv_heads, "active_units": n_active,
         "seq_lens": [int(v) for v in x.seq_lens.cpu().tolist()][:8],
-        "l2": "K/V caches larger than L2, and L2 flushed before every step by reading a 256 MiB buffer "
-              "(outside the per-step events)",
+        "l2": f"inputs larger than L2: the steps rotate over {n_input_sets(x)} independently seeded input sets "
+              f"({n_input_sets(x) * x.k_cache.numel() * 4 / 2**30:.2f} GiB of K/V), no flush",
         "parallelism": f"replicas x{n_gpus} (independent layer-steps, no collective on the data path)",
     }
 
@@ -260,6 +265,7 @@ def _captured_steps(native, dec, x, tau, steps, flush, split_events, fused, rota
                     ev[i][1].record(st)
                 native.decode_attention(*args, dec.active_list, dec.out, 0, dec.workspace)
             ev[i][2].record(st)
+    g.sr_events = ev  # recorded on every replay: they must live as long as the graph
     return g, ev
 
 
@@ -276,6 +282,55 @@ def time_steps(native, dec, x, tau, steps, warmup, flush, barrier, fused, rotate
     torch.cuda.synchronize()
     barrier()
     return [e[0].elapsed_time(e[2]) for e in ev]
+
+
+def time_back_to_back(native, dec, xs, tau, steps, warmup, fused=False, barrier=lambda: None):
+    """K layer-steps back to back in one CUDA graph, cycling over the input sets
+    `xs` (together larger than L2, so no flush is needed), timed as a block by
+    one event pair: (total ms, steps). This is how a decode forward runs its
+    layers; each step's launch overlaps the previous step's tail through the
+    programmatic dependency."""
+    import torch
+    dev = xs[0].q.device
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for xi in xs:
+            dec.step(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, tau)
+            dec.step_fused(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, tau)
+    torch.cuda.current_stream(dev).wait_stream(side)
+
+    def capture(n):
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            st = torch.cuda.current_stream()
+            e0.record(st)
+            for i in range(n):
+                xi = xs[i % len(xs)]
+                args = (xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens)
+                if fused:
+                    native.route_decode_attention(*args, tau, dec.out, dec.route_mask, dec.active_list, 0,
+                                                  dec.workspace)
+                else:
+                    native.route(xi.q, xi.k0, tau, dec.route_mask, dec.active_list)
+                    native.decode_attention(*args, dec.active_list, dec.out, 0, dec.workspace)
+            e1.record(st)
+        # the graph records these events on every replay: they must live as
+        # long as the graph
+        g.sr_events = (e0, e1)
+        return g, e0, e1
+
+    gw = capture(max(warmup, len(xs)))[0]
+    g, e0, e1 = capture(steps)
+    gw.replay()
+    barrier()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1), steps
 
 
 def time_kernels(native, dec, x, tau, steps, flush):
@@ -349,6 +404,7 @@ def _captured_append_steps(native, dec, x, a, tau, steps, flush, split_events):
             native.decode_attention(dec.q, x.k_cache, x.v_cache, x.k0, x.v0, a.seq_lens, dec.active_list, dec.out,
                                     0, dec.workspace)
             ev[i][2].record(st)
+    g.sr_events = ev  # recorded on every replay: they must live as long as the graph
     return g, ev
 
 
@@ -371,23 +427,64 @@ def time_append(native, dec, x, a, steps, warmup):
     return steps_ms, pre_ms
 
 
-def measure_config(native, inputs, name, steps, warmup, flush, device, peak, l2_mode="flush", copies=1):
-    """Routed and routing-disabled two-call steps of one more workload, for the
-    other_configs block. l2_mode: "flush" (a 256 MiB read before every step),
-    "hot" (no flush, the same inputs every step) or "rotate" (no flush; the
-    steps cycle over `copies` independently seeded input sets whose caches
-    together exceed L2)."""
+def measure_config(native, inputs, name, steps, warmup, flush, device, peak, l2_mode="rotate", copies=None,
+                   label=None, **kw):
+    """Routed and routing-disabled two-call steps and the fused launch of one more
+    workload, K steps back to back per graph. l2_mode: "hot" (the same inputs
+    every step, L2-resident when small) or "rotate" (the steps cycle over
+    independently seeded input sets whose caches together exceed three times
+    L2; `copies` overrides their number)."""
     import torch
-    xs = [inputs.make(name, seed=100 + c, device=device) for c in range(copies if l2_mode == "rotate" else 1)]
+    if l2_mode == "hot":
+        xs = [inputs.make(name, seed=100, device=device, **kw)]
+    elif copies:
+        xs = [inputs.make(name, seed=100 + 7919 * c, device=device, **kw) for c in range(copies)]
+    else:
+        xs = input_sets(inputs, name, 100, device, **kw)
     x = xs[0]
-    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=device)
-    fl = flush if l2_mode == "flush" else None
-    rot = xs if l2_mode == "rotate" else None
     nobar = lambda: None  # noqa: E731
-    routed = time_steps(native, dec, x, x.tau, steps, warmup, fl, nobar, False, rot)
-    disabled = time_steps(native, dec, x, float("inf"), steps, warmup, fl, nobar, False, rot)
-    if dec.workspace.device_error():
-        raise RuntimeError(f"device error word set on {name}")
+    r = measure_workload(native, inputs, xs, steps, warmup, flush, nobar, fused=True, isolated=False)
+    us, us_dis = r["block"] / steps * 1e3, r["block_disabled"] / steps * 1e3
+    us_f, us_fd = r["block_fused"] / steps * 1e3, r["block_fused_disabled"] / steps * 1e3
+    need, need_all = r["need"], r["need_all"]
+    gbs = need / (us * 1e-6) / 1e9
+    acts = [len(a) for a in r["actives"]]
+    out = {"workload": label or name, "context": x.max_seq_len,
+           "l2": "hot (one input set)" if l2_mode == "hot" else
+           f"rotate over {len(xs)} input sets ({len(xs) * x.k_cache.numel() * 4 / 2**30:.2f} GiB of K/V)",
+           "us_per_layer_step": round(us, 3), "needed_bytes": int(need), "effective_gbs": round(gbs, 1),
+           "frac_of_hbm_peak": round(gbs / peak, 4),
+           "active_units": acts[0] if len(set(acts)) == 1 else acts, "units": x.batch * x.n_kv_heads,
+           "routing_disabled_us": round(us_dis, 3),
+           "routing_disabled_gbs": round(need_all / (us_dis * 1e-6) / 1e9, 1),
+           "speedup_routed": round(us_dis / us, 3),
+           "fused_us": round(us_f, 3), "fused_disabled_us": round(us_fd, 3),
+           "fused_speedup_routed": round(us_fd / us_f, 3)}
+    del xs, x, r
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_workload(native, inputs, xs, steps, warmup, flush, barrier, fused=True, isolated=True):
+    """Timings of one workload on this GPU. `xs` are input sets of the workload
+    (xs[0] the main one) that together exceed L2.
+
+    block*: K layer-steps back to back in one graph over the input sets, one
+    event pair around all of them (ms in total): two-call routed and disabled,
+    and, if asked, the fused launch routed and disabled.
+    two*/route/decode (isolated=True): every step on its own between two events
+    after an L2 flush, on xs[0] (ms per step), and the two kernels' own times."""
+    import torch
+    x = xs[0]
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
+    for _ in range(warmup):
+        for xi in xs:
+            dec.step(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, xi.tau)
+            dec.step_fused(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, xi.tau)
+    torch.cuda.synchronize()
+    err = dec.workspace.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err} after warm-up")
     needs, needs_all, acts = [], [], []
     for xi in xs:
         dec.step(xi.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, xi.seq_lens, xi.tau)
@@ -396,48 +493,43 @@ def measure_config(native, inputs, name, steps, warmup, flush, device, peak, l2_
         needs.append(inputs.needed_bytes(sl, act, xi.n_kv_heads, xi.n_q_heads, xi.batch))
         needs_all.append(inputs.needed_bytes(sl, range(xi.batch * xi.n_kv_heads), xi.n_kv_heads, xi.n_q_heads,
                                              xi.batch))
-        acts.append(len(act))
-    need, need_all = statistics.mean(needs), statistics.mean(needs_all)
-    us, us_dis = statistics.mean(routed) * 1e3, statistics.mean(disabled) * 1e3
-    gbs = need / (us * 1e-6) / 1e9
-    gbs_dis = need_all / (us_dis * 1e-6) / 1e9
-    out = {"workload": name, "l2": l2_mode + (f" over {copies} input sets" if l2_mode == "rotate" else ""),
-           "us_per_layer_step": round(us, 3), "us_p50": round(statistics.median(routed) * 1e3, 3),
-           "needed_bytes": int(need), "effective_gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peak, 4),
-           "active_units": acts[0] if len(set(acts)) == 1 else acts, "units": x.batch * x.n_kv_heads,
-           "routing_disabled_us": round(us_dis, 3), "routing_disabled_gbs": round(gbs_dis, 1),
-           "speedup_routed": round(us_dis / us, 3)}
-    del xs, x, dec
-    torch.cuda.empty_cache()
-    return out
-
-
-def measure_workload(native, inputs, x, steps, warmup, flush, barrier, fused=True):
-    """Timings of one workload on this GPU: the two-call step (routed and with
-    routing disabled) and its kernels, and, if asked, the fused step."""
-    import torch
-    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len, device=x.q.device)
-    for _ in range(warmup):
-        dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
-        dec.step_fused(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
-    torch.cuda.synchronize()
-    err = dec.workspace.device_error()
-    if err:
-        raise RuntimeError(f"device error word {err} after warm-up")
-    act = active_units_of(dec.active_list.cpu())
-    sl = x.seq_lens.cpu().tolist()
-    r = dict(dec=dec, active=act, need=inputs.needed_bytes(sl, act, x.n_kv_heads, x.n_q_heads, x.batch),
-             need_all=inputs.needed_bytes(sl, range(x.batch * x.n_kv_heads), x.n_kv_heads, x.n_q_heads, x.batch))
-    r["two"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, False)
-    r["route"], r["decode"] = time_kernels(native, dec, x, x.tau, steps, flush)
-    r["two_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, False)
+        acts.append(act)
+    # the byte counts of the block are the mean over the rotated sets; the
+    # isolated steps run on xs[0]
+    r = dict(dec=dec, active=acts[0], actives=acts, need=statistics.mean(needs),
+             need_all=statistics.mean(needs_all), need0=needs[0], need_all0=needs_all[0])
+    x_tau = x.tau
+    r["block"] = time_back_to_back(native, dec, xs, x_tau, steps, warmup, False, barrier)[0]
+    r["block_disabled"] = time_back_to_back(native, dec, xs, float("inf"), steps, warmup, False, barrier)[0]
     if fused:
-        r["fused"] = time_steps(native, dec, x, x.tau, steps, warmup, flush, barrier, True)
-        r["fused_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, True)
+        r["block_fused"] = time_back_to_back(native, dec, xs, x_tau, steps, warmup, True, barrier)[0]
+        r["block_fused_disabled"] = time_back_to_back(native, dec, xs, float("inf"), steps, warmup, True,
+                                                      barrier)[0]
+    if isolated:
+        r["two"] = time_steps(native, dec, x, x_tau, steps, warmup, flush, barrier, False)
+        r["route"], r["decode"] = time_kernels(native, dec, x, x_tau, steps, flush)
+        r["two_disabled"] = time_steps(native, dec, x, float("inf"), steps, warmup, flush, barrier, False)
+        if fused:
+            r["fused"] = time_steps(native, dec, x, x_tau, steps, warmup, flush, barrier, True)
     err = dec.workspace.device_error()
     if err:
         raise RuntimeError(f"device error word {err} after the timed steps")
     return r
+
+
+def n_input_sets(x, min_bytes=3 * (126 << 20), max_sets=32) -> int:
+    """Input sets to rotate over for workload x: at least three, and as many as
+    it takes for their K/V caches together to exceed `min_bytes` (three times
+    L2), so that no step finds its inputs in L2."""
+    per_set = x.k_cache.numel() * 2 * 2
+    return max(3, min(max_sets, -(-min_bytes // per_set)))
+
+
+def input_sets(inputs, name, seed, device, **kw):
+    """n_input_sets independently seeded input sets of one workload."""
+    xs = [inputs.make(name, seed=seed, device=device, **kw)]
+    xs += [inputs.make(name, seed=seed + 7919 * c, device=device, **kw) for c in range(1, n_input_sets(xs[0]))]
+    return xs
 
 
 def e2e_measure(native, x, steps):
@@ -568,10 +660,16 @@ def e2e_append_graph_measure(native, x, a, steps):
     return e0.elapsed_time(e1) / steps
 
 
+def oracle_threads(n_active: int, group: int) -> int:
+    """Threads for the oracle: one per active (unit, query head) pair, capped
+    at the host cores."""
+    return max(1, min(os.cpu_count() or 1, max(1, n_active * group)))
+
+
 def oracle_layer_step_us(x_cpu, budget_s, min_reps=1, threads=None):
     """The fp64 oracle, as it stands, on whole layer-steps of this workload,
-    with `threads` threads (default: one per active unit, capped at the host
-    cores; the oracle splits whole units over its threads)."""
+    with `threads` threads (default: one per active (unit, query head) pair,
+    capped at the host cores; the oracle deals whole heads to its threads)."""
     import torch
 
     import oracle
@@ -579,7 +677,7 @@ def oracle_layer_step_us(x_cpu, budget_s, min_reps=1, threads=None):
     mask, active, _ = oracle.route(x_cpu.q, x_cpu.k0, tau)
     n_act = int(active[0])
     if threads is None:
-        threads = max(1, min(os.cpu_count() or 1, max(1, n_act)))
+        threads = oracle_threads(n_act, x_cpu.n_q_heads // x_cpu.n_kv_heads)
     reps = 0
     t0 = time.perf_counter()
     while True:
@@ -621,37 +719,41 @@ def run_ours(args):
     # fp32 so that torch sums it in place (a pure 256 MiB read; integer sums would
     # first widen the buffer with a 2 GB write).
     flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    x = inputs.make(args.config, seed=args.seed + 1000 * rank, device=dev)
+    # three (or more) independently seeded input sets whose caches together
+    # exceed L2: the timed steps rotate over them, so no step finds its K/V in L2
+    xs = input_sets(inputs, args.config, args.seed + 1000 * rank, dev)
+    x = xs[0]
     clocks = ClockSampler(local)
     clocks.start()
     t_wall = time.perf_counter()
-    r = measure_workload(native, inputs, x, args.steps, args.warmup, flush, barrier)
+    r = measure_workload(native, inputs, xs, args.steps, args.warmup, flush, barrier)
     t_wall = time.perf_counter() - t_wall
     clk = clocks.stop()
 
     K = args.steps
-    sum_ms = max_over_ranks(sum(r["two"]))
-    us_step, value = aggregate_us(sum_ms, K, world)
-    us_dis, _ = aggregate_us(max_over_ranks(sum(r["two_disabled"])), K, world)
-    us_fused, _ = aggregate_us(max_over_ranks(sum(r["fused"])), K, world)
-    us_fused_dis, _ = aggregate_us(max_over_ranks(sum(r["fused_disabled"])), K, world)
+    us_step, value = aggregate_us(max_over_ranks(r["block"]), K, world)
+    us_dis, _ = aggregate_us(max_over_ranks(r["block_disabled"]), K, world)
+    us_fused, _ = aggregate_us(max_over_ranks(r["block_fused"]), K, world)
+    us_fused_dis, _ = aggregate_us(max_over_ranks(r["block_fused_disabled"]), K, world)
+    us_iso, _ = aggregate_us(max_over_ranks(sum(r["two"])), K, world)
+    us_iso_dis, _ = aggregate_us(max_over_ranks(sum(r["two_disabled"])), K, world)
+    us_iso_fused, _ = aggregate_us(max_over_ranks(sum(r["fused"])), K, world)
     step_p = [v * 1e3 for v in r["two"]]
     dec_us = statistics.mean(r["decode"]) * 1e3
     route_us = statistics.median(r["route"]) * 1e3
-    need = r["need"]
+    need, need0 = r["need"], r["need0"]
     gbs = lambda nbytes, us: nbytes / (us * 1e-6) / 1e9  # noqa: E731
-    achieved = gbs(need, dec_us)  # the decode kernel, timed alone
+    achieved = gbs(need0, dec_us)  # the decode kernel, timed alone on xs[0]
     traffic = profiled_traffic()
 
+    cfg = describe_config(x, len(r["active"]), world)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(us_step / 1e3, 6), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
-        "config": describe_config(x, len(r["active"]), world),
+        "config": cfg,
         "path": "sr_route then sr_decode_attention (decode launch overlaps routing: programmatic dependency)",
         "effective_gbs": round(gbs(need, us_step), 1), "frac_of_hbm_peak": round(gbs(need, us_step) / peak, 4),
-        "route_kernel_us_median": round(route_us, 3), "decode_kernel_us_mean": round(dec_us, 3),
-        "step_us_p10_p50_p90": [round(statistics.quantiles(step_p, n=10)[i], 3) for i in (0, 4, 8)],
         "needed_bytes_per_step": need,
         "routing_disabled": {"us_per_layer_step": round(us_dis, 3),
                              "effective_gbs": round(gbs(r["need_all"], us_dis), 1),
@@ -662,14 +764,24 @@ def run_ours(args):
                                 "us_per_layer_step": round(us_fused, 3),
                                 "effective_gbs": round(gbs(need, us_fused), 1),
                                 "routing_disabled_us": round(us_fused_dis, 3)},
+        "isolated_step": {
+            "note": "every step alone: L2 flush (a 256 MiB read), event, the step, event; on the first input set. "
+                    "Two empty kernels measure about 6 us in this protocol (event and launch latency)",
+            "us_per_layer_step": round(us_iso, 3),
+            "step_us_p10_p50_p90": [round(statistics.quantiles(step_p, n=10)[i], 3) for i in (0, 4, 8)],
+            "effective_gbs": round(gbs(need0, us_iso), 1), "frac_of_hbm_peak": round(gbs(need0, us_iso) / peak, 4),
+            "routing_disabled_us": round(us_iso_dis, 3), "speedup_routed": round(us_iso_dis / us_iso, 3),
+            "fused_us": round(us_iso_fused, 3),
+            "route_kernel_us_median": round(route_us, 3), "decode_kernel_us_mean": round(dec_us, 3)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": "decode_kernel<1,4> (persistent split-K scan + sink copy + merge)",
-                     "algorithmic_bytes_per_launch": need, "peak_source": f"{peak_kind} HBM copy"},
+                     "algorithmic_bytes_per_launch": need0, "peak_source": f"{peak_kind} HBM copy",
+                     "timing": "decode kernel alone: an event between the two kernels, after an L2 flush"},
         "gpu_launches": 2 * K,
-        "timing": "the K timed steps are captured in one CUDA graph (per step: L2 flush read, event, the "
-                  "step, event) and replayed once; the two-call figures come from the same protocol, and its "
-                  "per-kernel times from a graph with an event between the two kernels",
+        "timing": "value: the K timed layer-steps back to back in one CUDA graph (sr_route, sr_decode_attention, "
+                  "per step), one event pair around all of them, replayed once after a warm-up graph; the routing-"
+                  "disabled and fused figures use the same protocol",
         "clocks": clk,
         "timed_wall_s": round(t_wall, 3),
         "impl": "ours",
@@ -689,41 +801,49 @@ def run_ours(args):
         "us_per_layer_step": round(us_app, 3),
         "prestep_kernel_us_median": round(statistics.median(pre_ms) * 1e3, 3),
         "active_units": int(dec_a.active_list[0]),
-        "two_call_us_per_layer_step": round(us_step, 3)}
+        "two_call_isolated_us_per_layer_step": round(us_iso, 3),
+        "timing": "isolated steps (L2 flush, event, the two launches, event), as isolated_step"}
     del dec_a
     if world == 1 and not args.no_sweep:
         sweep = []
+        ks = max(20, min(K, 50))
         for frac in (0.0, 0.25, 0.5, 0.75, 1.0):
-            x5 = inputs.make("llama8b_512k", seed=args.seed, device=dev, sink_fraction=frac)
-            s5 = measure_workload(native, inputs, x5, max(20, min(K, 50)), args.warmup, flush, barrier,
-                                  fused=False)
-            u5 = statistics.mean(s5["two"]) * 1e3
-            ud5 = statistics.mean(s5["two_disabled"]) * 1e3
+            x5 = input_sets(inputs, "llama8b_512k", args.seed, dev, sink_fraction=frac)
+            s5 = measure_workload(native, inputs, x5, ks, args.warmup, flush, barrier, fused=False)
+            u5 = s5["block"] / ks * 1e3
+            ud5 = s5["block_disabled"] / ks * 1e3
             d5 = statistics.mean(s5["decode"]) * 1e3
             sweep.append({"sink_fraction": frac, "us_per_layer_step": round(u5, 2),
                           "effective_gbs": round(s5["need"] / (u5 * 1e-6) / 1e9, 1),
                           "frac_of_peak": round(s5["need"] / (u5 * 1e-6) / 1e9 / peak, 4),
-                          "decode_kernel_gbs": round(s5["need"] / (d5 * 1e-6) / 1e9, 1),
-                          "routing_disabled_us": round(ud5, 2), "speedup_routed": round(ud5 / u5, 3)})
+                          "decode_kernel_gbs": round(s5["need0"] / (d5 * 1e-6) / 1e9, 1),
+                          "routing_disabled_us": round(ud5, 2), "speedup_routed": round(ud5 / u5, 3),
+                          "isolated_us": round(statistics.mean(s5["two"]) * 1e3, 2),
+                          "isolated_disabled_us": round(statistics.mean(s5["two_disabled"]) * 1e3, 2)})
             del x5, s5
             torch.cuda.empty_cache()
         line["sweep_512k"] = sweep
     if world == 1 and not args.no_sweep:
-        # The remaining workloads: tiny 4K with L2 hot and cold (rotating over
-        # input sets that together exceed L2), the 128K layer rotating over
-        # three input sets instead of flushing, the ragged 70B-shaped and the
-        # LLaVA-shaped layers with the flush protocol.
+        # The remaining workloads (K steps back to back per graph): tiny 4K with
+        # L2 hot and with its inputs rotated beyond L2, the ragged 70B-shaped and
+        # the LLaVA-shaped layers.
         oc_steps = max(20, min(K, 50))
         line["other_configs"] = [
             measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "hot"),
-            measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "rotate", copies=12),
-            # the headline workload with the other valid L2 protocol: three
-            # independent layer inputs in rotation, each step streaming 268 MB
-            measure_config(native, inputs, "llama8b_128k", oc_steps, args.warmup, flush, dev, peak, "rotate",
-                           copies=3),
+            measure_config(native, inputs, "tiny_4k", oc_steps, args.warmup, flush, dev, peak, "rotate"),
             measure_config(native, inputs, "llama70b_ragged", oc_steps, args.warmup, flush, dev, peak),
             measure_config(native, inputs, "llava7b_mha", oc_steps, args.warmup, flush, dev, peak),
         ]
+        # Short contexts: the 8B-shaped layer (4 of 8 groups sinks) from 4K to
+        # 64K, two-call and fused, routed and disabled, inputs rotated beyond L2.
+        short = [measure_config(native, inputs, "llama8b_128k", oc_steps, args.warmup, flush, dev, peak,
+                                label=f"llama8b_{c // 1024}k", max_ctx=c)
+                 for c in (4096, 8192, 16384, 32768, 65536)]
+        faster = ["fused" if e["fused_us"] < e["us_per_layer_step"] else "two-call" for e in short]
+        line["short_context"] = {
+            "points": short,
+            "faster_path": dict(zip([e["workload"] for e in short], faster)),
+            "speedup_routed_two_call": {e["workload"]: e["speedup_routed"] for e in short}}
     if not args.no_e2e:
         ms, h2d, d2h = e2e_measure(native, x, args.e2e_steps)
         ms = max_over_ranks(ms)
@@ -755,7 +875,8 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"{reps} whole layer-steps of {x.workload.name} "
                                           f"({x.batch * x.n_kv_heads} units) in {el:.1f} s, fp64 C oracle, "
-                                          f"{threads} threads (one per active unit, capped at the host cores)",
+                                          f"{threads} threads (one per active (unit, query head) pair, capped "
+                                          f"at the host cores)",
                                 "host_cores": os.cpu_count(),
                                 "one_thread": {"value": round(us1, 1), "unit": UNIT,
                                                "sample": f"{reps1} layer-steps in {el1:.1f} s"}}
@@ -781,7 +902,7 @@ def run_reference(args):
     import oracle
     mask, active, _ = oracle.route(x.q, x.k0, tau)
     n_act = int(active[0])
-    threads = max(1, min(os.cpu_count() or 1, max(1, n_act)))
+    threads = oracle_threads(n_act, x.n_q_heads // x.n_kv_heads)
     # Each step is one whole layer-step unless that would make the run exceed
     # about three minutes; then a step is a bounded sample of the active units,
     # scaled to the whole layer-step.
@@ -811,13 +932,36 @@ def run_reference(args):
         "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": describe_config(x, n_act, 1) | {"parallelism": "host cores (CPU oracle)"},
+        "config": describe_config(x, n_act, world),
         "impl": "reference",
         "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": sample, "host_cores": os.cpu_count()},
+                         "sample": sample + f", fp64 C oracle on {threads} host threads (one per active "
+                                            f"(unit, query head) pair, capped at the host cores)",
+                         "host_cores": os.cpu_count()},
         "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_profile(args):
+    """A few eager two-call steps of one workload, for profiler captures: no
+    timing, no flush, few launches before the captured ones."""
+    import torch
+
+    from kv_cache_routing_sr_b200 import inputs, native
+    x = inputs.make(args.profile, seed=args.seed, device="cuda", max_ctx=args.max_ctx)
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    for _ in range(args.warmup + args.steps):
+        dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, x.tau)
+    torch.cuda.synchronize()
+    if dec.workspace.device_error():
+        raise RuntimeError(f"device error word {dec.workspace.device_error()}")
+    act = active_units_of(dec.active_list.cpu())
+    need = inputs.needed_bytes(x.seq_lens.cpu().tolist(), act, x.n_kv_heads, x.n_q_heads, x.batch)
+    print(json.dumps({"profile": args.profile, "batch": x.batch, "context": x.max_seq_len,
+                      "q_heads": x.n_q_heads, "kv_heads": x.n_kv_heads, "active_units": len(act),
+                      "units": x.batch * x.n_kv_heads, "needed_bytes_per_step": need,
+                      "steps": args.warmup + args.steps, "launches_per_step": 2}))
 
 
 def run_multilayer(args):
@@ -976,6 +1120,8 @@ def main(argv=None):
     if args.proxy_quality:
         run_proxy_quality(args)
         return
+    if args.profile:
+        return run_profile(args)
     if args.multilayer:
         run_multilayer(args)
         return
