@@ -775,7 +775,7 @@ def run_ours(args):
             "route_kernel_us_median": round(route_us, 3), "decode_kernel_us_mean": round(dec_us, 3)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "decode_kernel<1,4> (persistent split-K scan + sink copy + merge)",
+                     "kernel": "decode_kernel<2,2> (persistent split-K scan + sink copy + merge)",
                      "algorithmic_bytes_per_launch": need0, "peak_source": f"{peak_kind} HBM copy",
                      "timing": "decode kernel alone: an event between the two kernels, after an L2 flush"},
         "gpu_launches": 2 * K,

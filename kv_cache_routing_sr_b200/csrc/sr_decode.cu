@@ -49,14 +49,25 @@
 #include "sr_route_math.cuh"
 #include "sr_timeline.cuh"
 
+// Two row blocks of 16 per consumer warp (128-row tiles) in two 64 KB stages:
+// the same 128 KB in flight per SM as four 64-row stages, with two independent
+// MMA chains per warp. Measured back to back at 128K: 49.6-50.0 us per
+// layer-step against 50.7 for RB = 1 with four stages (and 52.4 for RB = 2
+// with three stages, 192 KB in flight).
 #ifndef SR_DECODE_RB
-#define SR_DECODE_RB 1 // row blocks of 16 per consumer warp and tile
+#define SR_DECODE_RB 2 // row blocks of 16 per consumer warp and tile
 #endif
 #ifndef SR_DECODE_STAGES
-#define SR_DECODE_STAGES 4
+#define SR_DECODE_STAGES 2
 #endif
 
 SR_TL_DEFINE(tl_decode)
+#ifdef SR_TIMELINE
+// latest %globaltimer at which a decode CTA left (atomicMax); the next kernel
+// reads it after its dependency wait
+static __device__ unsigned long long tl_last_exit;
+extern "C" int sr_timeline_last_exit_addr(void **p) { return (int)cudaGetSymbolAddress(p, tl_last_exit); }
+#endif
 
 namespace sr {
 namespace {
@@ -330,6 +341,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         grid_launch_dependents();
         if (tid == 0)
             SR_STAMP(tl_decode, 1);
+#ifdef SR_TIMELINE
+        if (tid == 0 && blockIdx.x < SR_TL_CTAS)
+            tl_decode[blockIdx.x][15] = *(volatile unsigned long long *)&tl_last_exit;
+#endif
         // All inputs are read after the wait: the preceding kernel may write
         // any of them (the routing kernel the list, the append step seq_lens).
         const int sl = (lane < p.B) ? __ldg(p.seq_lens + lane) : 1;
@@ -1075,6 +1090,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         atomicOr(p.err, SR_DEVERR_TIMEOUT);
 #ifdef SR_TIMELINE
     if (ctid == 0) {
+        unsigned long long t_;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));
+        atomicMax(&tl_last_exit, t_);
         SR_STAMP(tl_decode, 11);
         tl_decode[blockIdx.x][12] = (unsigned long long)tl_splits;
         tl_decode[blockIdx.x][13] = (unsigned long long)tl_last;

@@ -27,6 +27,11 @@
 #include "sr_timeline.cuh"
 
 SR_TL_DEFINE(tl_route)
+#ifdef SR_TIMELINE
+// set by the host to the decode kernel's last-exit word (sr_timeline_last_exit_addr)
+static __device__ unsigned long long *tl_exit_ptr;
+extern "C" int sr_timeline_set_exit_ptr(void *p) { return (int)cudaMemcpyToSymbol(tl_exit_ptr, &p, sizeof(p)); }
+#endif
 
 namespace sr {
 namespace {
@@ -55,6 +60,10 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
     grid_launch_dependents();
     if (threadIdx.x == 0)
         SR_STAMP(tl_route, 1);
+#ifdef SR_TIMELINE
+    if (threadIdx.x == 0 && tl_exit_ptr)
+        tl_route[0][5] = *(volatile unsigned long long *)tl_exit_ptr;
+#endif
 
     route_units_warp<M, true>(reinterpret_cast<const uint4 *>(q), reinterpret_cast<const uint4 *>(k0), U, tau,
                               (int)threadIdx.x >> 5, kRouteWarps, [&](int u, bool sink) {
