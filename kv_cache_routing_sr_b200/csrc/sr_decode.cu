@@ -66,6 +66,7 @@ SR_TL_DEFINE(tl_decode)
 // latest %globaltimer at which a decode CTA left (atomicMax); the next kernel
 // reads it after its dependency wait
 static __device__ unsigned long long tl_last_exit;
+static __device__ unsigned int tl_decode_launch; // ring of CTA 0's stamps in rows 512 .. 575
 extern "C" int sr_timeline_last_exit_addr(void **p) { return (int)cudaGetSymbolAddress(p, tl_last_exit); }
 #endif
 
@@ -99,6 +100,19 @@ struct alignas(16) TileHdr {
 #define SR_DECODE_SEQTAB 4096
 #endif
 constexpr int kSeqTab = SR_DECODE_SEQTAB; // seq_lens entries staged in shared memory
+
+// Launches of at most kFastUnits units: the active entry of rank r, prepared by
+// lane r of the producer warp so that the producer lane reads its splits from a
+// table instead of deriving them one after another.
+struct alignas(16) RankInfo {
+    long long start; // prefix of the active lengths before this rank
+    int32_t unit;    // flat unit b*Hkv+g
+    int32_t len;     // length, clamped to [1, Lmax]
+    int32_t qrow;    // first query row of the unit, b*Hq + g*M
+    int32_t cf;      // automatic splits: first share overlapping the unit
+    int32_t cl;      // automatic splits: last share overlapping the unit
+    int32_t pad;
+};
 
 struct Misc {
     int abort_flag;
@@ -147,7 +161,8 @@ template <int RB, int STAGES> struct Cfg {
     // seq_lens staged outside the stage buffers: the producer reads it while
     // the copies run
     static constexpr int OFF_SEQ = OFF_BITMAP + SR_MAX_UNITS / 8;
-    static constexpr int BYTES = OFF_SEQ + kSeqTab * 4;
+    static constexpr int OFF_RANK = OFF_SEQ + kSeqTab * 4; // RankInfo[32] (launches of <= 32 units)
+    static constexpr int BYTES = OFF_RANK + 32 * (int)sizeof(RankInfo);
     static constexpr int ALLOC = BYTES + 1024; // room to align the base to 1024 B
     static_assert(sizeof(Misc) <= 256, "misc block");
     // Prologue tables (active lengths, active units, sink flags) live in the
@@ -319,6 +334,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     // kFastUnits units only).
     const bool seq_smem = p.B <= kSeqTab;
     int32_t *seqtab = reinterpret_cast<int32_t *>(smem + C::OFF_SEQ);
+    RankInfo *rtab = reinterpret_cast<RankInfo *>(smem + C::OFF_RANK);
     int32_t *ltab = reinterpret_cast<int32_t *>(smem);
     int16_t *utab = reinterpret_cast<int16_t *>(smem + ((4 * U + 127) & ~127));
     uint8_t *sflag = smem + ((4 * U + 127) & ~127) + ((2 * U + 127) & ~127);
@@ -344,6 +360,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 #ifdef SR_TIMELINE
         if (tid == 0 && blockIdx.x < SR_TL_CTAS)
             tl_decode[blockIdx.x][15] = *(volatile unsigned long long *)&tl_last_exit;
+        if (tid == 0 && blockIdx.x == 0) {
+            const unsigned int ring = 512 + atomicAdd(&tl_decode_launch, 1u) % 64u;
+            tl_decode[ring][1] = tl_decode[0][1];
+            tl_decode[ring][15] = tl_decode[0][15];
+        }
 #endif
         // All inputs are read after the wait: the preceding kernel may write
         // any of them (the routing kernel the list, the append step seq_lens).
@@ -523,6 +544,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 misc->s0 = s0;
                 misc->first_u = fu;
             }
+            if (lane < n) {
+                RankInfo ri;
+                ri.start = lane_incl - lane_len;
+                ri.unit = lane_unit;
+                ri.len = lane_len;
+                const int b = lane_unit / p.Hkv;
+                ri.qrow = b * p.Hq + (lane_unit - b * p.Hkv) * M;
+                ri.cf = (p.n_splits == 0) ? (int)div_nonneg(ri.start, chunk) : 0;
+                ri.cl = (p.n_splits == 0) ? (int)div_nonneg(ri.start + lane_len - 1, chunk) : 0;
+                ri.pad = 0;
+                rtab[lane] = ri;
+            }
             __syncwarp();
         }
     } else {
@@ -562,6 +595,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         if (lane != 0)
             return;
         const uint64_t pol = l2_policy_evict_first();
+        SR_STAMP(tl_decode, 16);
         int stage = 0;
         uint32_t ph = 0;
         int issued_parity[STAGES];
@@ -571,8 +605,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         bool ok = true;
 
         auto emit = [&](const TileHdr &h, const void *qsrc, uint32_t qbytes) -> bool {
+#ifdef SR_TIMELINE
+            const bool tl_first = issued_parity[stage] < 0 && stage == 0 && ph == 0;
+            if (tl_first)
+                SR_STAMP(tl_decode, 17);
+#endif
             if (!wait_bar(empty0 + 8 * stage, ph ^ 1, abort_flag))
                 return false;
+#ifdef SR_TIMELINE
+            if (tl_first)
+                SR_STAMP(tl_decode, 18);
+#endif
             hdr[stage] = h;
             const uint32_t fb = full0 + 8 * stage;
             const uint32_t bytes = (h.nvalid > 0 ? (uint32_t)C::STAGE : 0u) + qbytes;
@@ -580,6 +623,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 mbar_arrive_expect_tx(fb, bytes);
                 if (h.nvalid > 0) {
                     const uint32_t sb = smem_u32(smem + stage * C::STAGE);
+#ifdef SR_TIMELINE
+                    if (tl_first)
+                        SR_STAMP(tl_decode, 19);
+#endif
                     tma_load_3d(sb, &tmK, fb, 0, h.pos0, h.unit, pol);
                     tma_load_3d(sb + C::HALF, &tmK, fb, 64, h.pos0, h.unit, pol);
                     tma_load_3d(sb + 2 * C::HALF, &tmV, fb, 0, h.pos0, h.unit, pol);
@@ -600,11 +647,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             return true;
         };
 
-        auto emit_split = [&](int u, long long b0, long long e0, int slot, int nseg, int slot_first) -> bool {
+        auto emit_split = [&](int u, int qrow, long long b0, long long e0, int slot, int nseg,
+                              int slot_first) -> bool {
             const long long len = e0 - b0;
             const long long ntiles = len > 0 ? (len + C::BN - 1) / C::BN : 1;
-            const int sb = u / p.Hkv, sg = u - sb * p.Hkv;
-            const __nv_bfloat16 *qsrc = p.q + ((size_t)sb * p.Hq + (size_t)sg * M) * kHeadDim;
+            const __nv_bfloat16 *qsrc = p.q + (size_t)qrow * kHeadDim;
+#ifdef SR_TIMELINE
+            if (issued_parity[0] < 0)
+                SR_STAMP(tl_decode, 21);
+#endif
             for (long long t = 0; t < ntiles; ++t) {
                 TileHdr h;
                 h.unit = u;
@@ -626,6 +677,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         // Active entry of rank i, for non-decreasing i: ranks follow the set
         // bits of the bitmap in ascending unit order, starting at first_u.
         int wi = misc->i0, wu = misc->first_u;
+        SR_STAMP(tl_decode, 22);
         auto unit_at = [&](int i) -> int {
             while (wi < i && wu < U) {
                 wu = next_set_bit(bitmap, wu + 1, U);
@@ -633,20 +685,54 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             }
             return wu;
         };
+        // Active entry of rank i (non-decreasing i) whose positions start at S:
+        // from the rank table when the launch has at most kFastUnits units,
+        // else from the bitmap walk and the length table. u < 0 ends the walk.
+        struct Rank {
+            int u, L, qrow;
+            long long cf, cl;
+        };
+        auto rank_at = [&](int i, long long S) -> Rank {
+            Rank r;
+            if (fast) {
+                const RankInfo ri = rtab[i];
+                r.u = ri.unit;
+                r.L = ri.len;
+                r.qrow = ri.qrow;
+                r.cf = ri.cf;
+                r.cl = ri.cl;
+                return r;
+            }
+            r.u = unit_at(i);
+            if (r.u < 0 || r.u >= U) {
+                r.u = -1;
+                return r;
+            }
+            r.L = unit_len(p, r.u, seq_smem ? seqtab : nullptr);
+            const int b = r.u / p.Hkv;
+            r.qrow = b * p.Hq + (r.u - b * p.Hkv) * M;
+            if (p.n_splits == 0) {
+                r.cf = div_nonneg(S, chunk);
+                r.cl = div_nonneg(S + r.L - 1, chunk);
+            }
+            return r;
+        };
         if (p.n_splits == 0) {
             if (P > 0 && r0 < P) {
                 int i = misc->i0;
                 long long S = misc->s0;
                 while (ok && i < n && S < r1) {
-                    const int u = unit_at(i);
-                    if (u < 0 || u >= U)
+                    const Rank r = rank_at(i, S);
+                    if (r.u < 0)
                         break;
-                    const int L = unit_len(p, u, seq_smem ? seqtab : nullptr);
                     const long long b0 = (r0 > S ? r0 : S) - S;
-                    const long long e0 = (r1 < S + L ? r1 : S + L) - S;
-                    const long long cf = div_nonneg(S, chunk), cl = div_nonneg(S + L - 1, chunk);
-                    ok = emit_split(u, b0, e0, (int)blockIdx.x + i, (int)(cl - cf + 1), (int)cf + i);
-                    S += L;
+                    const long long e0 = (r1 < S + r.L ? r1 : S + r.L) - S;
+#ifdef SR_TIMELINE
+                    if (i == misc->i0)
+                        SR_STAMP(tl_decode, 20);
+#endif
+                    ok = emit_split(r.u, r.qrow, b0, e0, (int)blockIdx.x + i, (int)(r.cl - r.cf + 1), (int)r.cf + i);
+                    S += r.L;
                     ++i;
                 }
             }
@@ -654,12 +740,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             const int ns = p.n_splits;
             for (long long j = blockIdx.x; ok && j < (long long)n * ns; j += G) {
                 const int i = (int)div_nonneg(j, ns), s = (int)(j - (long long)i * ns);
-                const int u = unit_at(i);
-                if (u < 0 || u >= U)
+                const Rank r = rank_at(i, 0);
+                if (r.u < 0)
                     break;
-                const int L = unit_len(p, u, seq_smem ? seqtab : nullptr);
-                const long long b0 = (long long)s * L / ns, e0 = (long long)(s + 1) * L / ns;
-                ok = emit_split(u, b0, e0, (int)j, ns, i * ns);
+                const long long b0 = (long long)s * r.L / ns, e0 = (long long)(s + 1) * r.L / ns;
+                ok = emit_split(r.u, r.qrow, b0, e0, (int)j, ns, i * ns);
             }
         }
         if (ok) {

@@ -30,6 +30,7 @@ SR_TL_DEFINE(tl_route)
 #ifdef SR_TIMELINE
 // set by the host to the decode kernel's last-exit word (sr_timeline_last_exit_addr)
 static __device__ unsigned long long *tl_exit_ptr;
+static __device__ unsigned int tl_route_launch; // ring of per-launch stamps in rows 1 .. 64
 extern "C" int sr_timeline_set_exit_ptr(void *p) { return (int)cudaMemcpyToSymbol(tl_exit_ptr, &p, sizeof(p)); }
 #endif
 
@@ -61,8 +62,14 @@ route_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restric
     if (threadIdx.x == 0)
         SR_STAMP(tl_route, 1);
 #ifdef SR_TIMELINE
-    if (threadIdx.x == 0 && tl_exit_ptr)
-        tl_route[0][5] = *(volatile unsigned long long *)tl_exit_ptr;
+    if (threadIdx.x == 0) {
+        const unsigned long long pe = tl_exit_ptr ? *(volatile unsigned long long *)tl_exit_ptr : 0ull;
+        tl_route[0][5] = pe;
+        const unsigned int ring = 1 + atomicAdd(&tl_route_launch, 1u) % 64u;
+        tl_route[ring][1] = tl_route[0][1];
+        tl_route[ring][5] = pe;
+        tl_route[ring][0] = tl_route[0][0];
+    }
 #endif
 
     route_units_warp<M, true>(reinterpret_cast<const uint4 *>(q), reinterpret_cast<const uint4 *>(k0), U, tau,
