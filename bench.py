@@ -43,6 +43,7 @@ METRIC = "decode-attention µs/layer-step and effective HBM GB/s (% of peak) at 
 UNIT = "us/layer-step"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the copy bandwidth above is the roofline)
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_128k.md")
 DECODE_SOURCE = os.path.join(ROOT, "kv_cache_routing_sr_b200", "csrc", "sr_decode.cu")
 L2_FLUSH_BYTES = 256 << 20
@@ -769,6 +770,7 @@ def run_ours(args):
         "config": cfg,
         "path": "sr_route then sr_decode_attention (decode launch overlaps routing: programmatic dependency)",
         "effective_gbs": round(gbs(need, us_step), 1), "frac_of_hbm_peak": round(gbs(need, us_step) / peak, 4),
+        "frac_of_nominal_hbm": round(gbs(need, us_step) / NOMINAL_HBM_GBS, 4),
         "needed_bytes_per_step": need,
         "routing_disabled": {"us_per_layer_step": round(us_dis, 3),
                              "effective_gbs": round(gbs(r["need_all"], us_dis), 1),
