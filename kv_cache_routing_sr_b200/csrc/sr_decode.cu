@@ -82,6 +82,13 @@ constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeThreads = 32 * kCWarps;
 constexpr int kMergeBatch = 16; // partials in flight per thread in the final merge
+// Row stride (floats) of the split-end scratch that holds each warp's O per
+// head: 4 floats of padding put the lanes that store the same row of
+// different head pairs in different banks.
+constexpr int kCombStride = 128 + 4;
+// Bytes per query head in the shared q buffer: the 256-byte row plus 16 bytes,
+// so the lanes that read the same word of different heads hit different banks.
+constexpr int kQRowBytes = kHeadDim * 2 + 16;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kFastUnits = 32; // launches with at most this many units plan in registers
 
@@ -150,10 +157,10 @@ template <int RB, int STAGES> struct Cfg {
     static constexpr int BN = 16 * RB * kCWarps; // positions per tile
     static constexpr int HALF = BN * 128;        // one [BN x 64] bf16 box
     static constexpr int STAGE = 4 * HALF;       // K lo, K hi, V lo, V hi
-    static constexpr int QBYTES = kMaxGroup * kHeadDim * 2;
+    static constexpr int QBYTES = kMaxGroup * kQRowBytes;
     static constexpr int OFF_Q = STAGES * STAGE;
     static constexpr int OFF_COMB = OFF_Q + STAGES * QBYTES;
-    static constexpr int OFF_ML = OFF_COMB + kCWarps * kMaxGroup * kHeadDim * 4;
+    static constexpr int OFF_ML = OFF_COMB + kCWarps * kMaxGroup * kCombStride * 4;
     static constexpr int OFF_HDR = OFF_ML + kCWarps * kMaxGroup * 8;
     static constexpr int OFF_BAR = OFF_HDR + STAGES * (int)sizeof(TileHdr);
     static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
@@ -632,8 +639,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     tma_load_3d(sb + 2 * C::HALF, &tmV, fb, 0, h.pos0, h.unit, pol);
                     tma_load_3d(sb + 3 * C::HALF, &tmV, fb, 64, h.pos0, h.unit, pol);
                 }
+                // the group's q rows, one copy per head into the padded rows
                 if (qbytes)
-                    bulk_load(smem_u32(smem + C::OFF_Q + stage * C::QBYTES), qsrc, qbytes, fb);
+                    for (int hq = 0; hq < M; ++hq)
+                        bulk_load(smem_u32(smem + C::OFF_Q + stage * C::QBYTES + hq * kQRowBytes),
+                                  static_cast<const uint8_t *>(qsrc) + hq * kHeadDim * 2, kHeadDim * 2, fb);
                 if (issued_parity[stage] < 0 && stage == 0 && ph == 0)
                     SR_STAMP(tl_decode, 4);
                 issued_parity[stage] = (int)ph;
@@ -874,8 +884,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 const uint32_t *qs = reinterpret_cast<const uint32_t *>(smem + C::OFF_Q + stage * C::QBYTES);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    qf[ks][0] = (g < M) ? qs[g * 64 + ks * 8 + t] : 0u;
-                    qf[ks][1] = (g < M) ? qs[g * 64 + ks * 8 + 4 + t] : 0u;
+                    qf[ks][0] = (g < M) ? qs[g * (kQRowBytes / 4) + ks * 8 + t] : 0u;
+                    qf[ks][1] = (g < M) ? qs[g * (kQRowBytes / 4) + ks * 8 + 4 + t] : 0u;
                 }
             }
         }
@@ -1001,17 +1011,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 mlsm[w * kMaxGroup + 2 * t + 1] = make_float2(mrun[1], l1);
             }
             // Unscaled O of this warp; the readers below weight the four warps.
-            float *cw = comb + w * (kMaxGroup * kHeadDim);
+            float *cw = comb + w * (kMaxGroup * kCombStride);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int d0 = 16 * j + g;
                 if (2 * t < M) {
-                    cw[(2 * t) * kHeadDim + d0] = o[j][0];
-                    cw[(2 * t) * kHeadDim + d0 + 8] = o[j][2];
+                    cw[(2 * t) * kCombStride + d0] = o[j][0];
+                    cw[(2 * t) * kCombStride + d0 + 8] = o[j][2];
                 }
                 if (2 * t + 1 < M) {
-                    cw[(2 * t + 1) * kHeadDim + d0] = o[j][1];
-                    cw[(2 * t + 1) * kHeadDim + d0 + 8] = o[j][3];
+                    cw[(2 * t + 1) * kCombStride + d0] = o[j][1];
+                    cw[(2 * t + 1) * kCombStride + d0 + 8] = o[j][3];
                 }
             }
             if (!(ok = cbar_sync()))
@@ -1035,7 +1045,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 for (int ww = 0; ww < kCWarps; ++ww) {
                     const float f = (ml[ww].x == -INFINITY) ? 0.f : exp2f(ml[ww].x - Mh);
                     const float4 x =
-                        *reinterpret_cast<const float4 *>(comb + ww * (kMaxGroup * kHeadDim) + head * kHeadDim + d4);
+                        *reinterpret_cast<const float4 *>(comb + ww * (kMaxGroup * kCombStride) + head * kCombStride + d4);
                     acc.x = fmaf(x.x, f, acc.x);
                     acc.y = fmaf(x.y, f, acc.y);
                     acc.z = fmaf(x.z, f, acc.z);
