@@ -385,6 +385,87 @@ class AppendInputs:
                                x.v0, self.seq_lens, tau)
 
 
+class AppendSequence:
+    """Inputs of `visits` consecutive append steps on workload x: visit t puts
+    the new token of every sequence at slot L - visits + t, so the last visit's
+    scan covers the full context; each visit's un-rotated query is the planted
+    query rotated back to its slot (by the library's own kernel), so routing
+    sees the same groups at every visit. reset() restores the lengths before a
+    graph replay."""
+
+    def __init__(self, native, inputs, x, visits):
+        import torch
+        dev = x.q.device
+        B, Hq, Hkv = x.batch, x.n_q_heads, x.n_kv_heads
+        self.seq_saved = (x.seq_lens - visits).clone()
+        self.seq_lens = self.seq_saved.clone()
+        self.cos, self.sin = inputs.rope_tables(x.max_seq_len, device=dev)
+        _, self.k_new, self.v_new = inputs.make_projections(B, Hq, Hkv, seed=x.seed + 17, device=dev)
+        z1 = torch.zeros((1, Hkv, 1, 128), dtype=torch.bfloat16, device=dev)
+        self.q_in = []
+        for t in range(visits):
+            q_in = torch.empty_like(x.q)
+            for b, p0 in enumerate(self.seq_saved.tolist()):
+                p = p0 + t
+                zr = torch.zeros((1, Hkv, 128), dtype=torch.bfloat16, device=dev)
+                native.rope_append_route(x.q[b:b + 1].contiguous(), zr, zr.clone(), self.cos[p:p + 1].contiguous(),
+                                         (-self.sin[p:p + 1]).contiguous(),
+                                         torch.zeros(1, dtype=torch.int32, device=dev), z1.clone(), z1.clone(),
+                                         zr.clone(), zr.clone(), float("inf"), q_out=q_in[b:b + 1])
+            self.q_in.append(q_in)
+        torch.cuda.synchronize()
+
+    def reset(self):
+        self.seq_lens.copy_(self.seq_saved)
+
+
+def time_append_back_to_back(native, dec, xs, seqs, tau, steps, warmup):
+    """K append steps (sr_rope_append_route, sr_decode_attention) back to back
+    in one CUDA graph, cycling over the input sets `xs` (each with its
+    AppendSequence in `seqs`), one event pair around all of them: total ms. The
+    lengths are restored outside the graph before each replay."""
+    import torch
+    dev = xs[0].q.device
+    if getattr(dec, "q", None) is None:
+        dec.q = torch.empty_like(xs[0].q)
+    n = len(xs)
+
+    def step(i):
+        xi, a = xs[i % n], seqs[i % n]
+        native.rope_append_route(a.q_in[i // n], a.k_new, a.v_new, a.cos, a.sin, a.seq_lens, xi.k_cache,
+                                 xi.v_cache, xi.k0, xi.v0, tau, dec.q, dec.route_mask, dec.active_list)
+        native.decode_attention(dec.q, xi.k_cache, xi.v_cache, xi.k0, xi.v0, a.seq_lens, dec.active_list, dec.out,
+                                0, dec.workspace)
+
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):  # eager warm-up outside the capture
+        for i in range(min(steps, n)):
+            step(i)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = torch.cuda.current_stream()
+        e0.record(st)
+        for i in range(steps):
+            step(i)
+        e1.record(st)
+    g.sr_events = (e0, e1)  # recorded on every replay: they must live as long as the graph
+    for _ in range(max(1, -(-warmup // steps))):  # untimed: warm-up and the graph's launch set-up
+        for a in seqs:
+            a.reset()
+        g.replay()
+    torch.cuda.synchronize()
+    for a in seqs:
+        a.reset()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
 def _captured_append_steps(native, dec, x, a, tau, steps, flush, split_events):
     """As _captured_steps for the append path: per step an L2 flush and the
     seq_lens reset, then an event, sr_rope_append_route, (an event,)
@@ -816,15 +897,24 @@ def run_ours(args):
     if dec_a.workspace.device_error():
         raise RuntimeError("device error word set by the append-step timing")
     us_app, _ = aggregate_us(max_over_ranks(sum(app_ms)), K, world)
+    # the same step back to back over the rotated input sets, as the headline
+    seqs = [AppendSequence(native, inputs, xi, -(-K // len(xs))) for xi in xs]
+    ms_b2b = time_append_back_to_back(native, dec_a, xs, seqs, x.tau, K, args.warmup)
+    if dec_a.workspace.device_error():
+        raise RuntimeError("device error word set by the back-to-back append-step timing")
+    us_app_b2b, _ = aggregate_us(max_over_ranks(ms_b2b), K, world)
     line["append_step"] = {
         "path": "sr_rope_append_route then sr_decode_attention (RoPE of the query heads and the new key, KV "
-                "append at the last slot, k0/v0 capture, routing and the length update in the first launch)",
-        "us_per_layer_step": round(us_app, 3),
+                "append, k0/v0 capture, routing and the length update in the first launch)",
+        "us_per_layer_step": round(us_app_b2b, 3),
+        "timing": "the K steps back to back in one CUDA graph over the rotated input sets (as value); each set's "
+                  "visits append at its last K/sets slots, the last visit at the final slot",
+        "isolated_us_per_layer_step": round(us_app, 3),
+        "isolated_two_call_us_per_layer_step": round(us_iso, 3),
+        "isolated_timing": "L2 flush, event, the two launches, event (as isolated_step), new token at the last slot",
         "prestep_kernel_us_median": round(statistics.median(pre_ms) * 1e3, 3),
-        "active_units": int(dec_a.active_list[0]),
-        "two_call_isolated_us_per_layer_step": round(us_iso, 3),
-        "timing": "isolated steps (L2 flush, event, the two launches, event), as isolated_step"}
-    del dec_a
+        "active_units": int(dec_a.active_list[0])}
+    del dec_a, seqs
     if world == 1 and not args.no_sweep:
         sweep = []
         ks = max(20, min(K, 50))

@@ -21,12 +21,12 @@
 // exponent, makes the double rounding innocuous; fp32 has sixteen more than
 // bf16). The result is the correctly rounded bf16 of the fp64 rotation.
 //
-// Layout: one CTA of 256 threads, like the routing kernel, walking the units
-// in chunks whose rows fit in shared memory. Per chunk: eight threads per new
-// key rotate it (each takes 8 elements and their 8 partners), write the cache
-// slot, and stage the group's position-0 key (the captured one at slot 0, else
-// the stored k0); eight threads per query row rotate it into q_out and the
-// staged rows; the staged rows are routed with the routing kernel's own
+// Layout: one CTA of 512 threads walking the units in chunks whose rows fit in
+// shared memory. Per chunk, in one pass where each thread takes its own item:
+// eight threads per new key rotate it (each takes 8 elements and their 8
+// partners), write the cache slot, and stage the group's position-0 key (the
+// captured one at slot 0, else the stored k0); eight threads per query row
+// rotate it into q_out and the staged rows; the staged rows are routed with the routing kernel's own
 // routine (one warp per GQA group), so the decision equals sr_route on
 // (q_out, k0) bit for bit. Lengths advance after every read of
 // them; the compaction is the routing kernel's.
@@ -42,7 +42,7 @@
 namespace sr {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 160 * 1024; // shared bytes for staged q / k0 rows
 
@@ -137,12 +137,45 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
     grid_dependency_wait();
     grid_launch_dependents();
 
+    // Query row item `it` of the chunk starting at unit u0: rotate into q_out and
+    // the staged rows; a sequence with no valid slot gets a zero query.
+    auto query_item = [&](int it, int u0) {
+        const int r = it >> 3, j = it & 7;
+        const int u = u0 + r / M;
+        const size_t row = ((size_t)u0 * M + r) * kHeadDim;
+        // plain loads: q_out may be q_in (rotated in place)
+        const uint4 *qi = reinterpret_cast<const uint4 *>(p.q_in + row);
+        const uint4 qlo = qi[j], qhi = qi[j + 8];
+        const int pos = slot_of(p, u / p.Hkv);
+        uint4 *qs = rows + r * 16;
+        uint4 *qd = reinterpret_cast<uint4 *>(p.q_out + row);
+        uint4 lo = zero, hi = zero;
+        if (pos >= 0) {
+            float4 c[2], s[2];
+            load_table8(p.rope_cos, pos, j, c);
+            load_table8(p.rope_sin, pos, j, s);
+            rope8(qlo, qhi, c, s, lo, hi);
+        }
+        qs[j] = lo;
+        qs[j + 8] = hi;
+        qd[j] = lo;
+        qd[j + 8] = hi;
+    };
+
     bool bad_slot = false;
     for (int u0 = 0; u0 < U; u0 += cu) {
         const int nu = (U - u0) < cu ? (U - u0) : cu;
         uint4 *krows = rows + (size_t)nu * M * 16;
-        // New key: rotate, append, capture or stage k0. New value: append.
-        for (int it = threadIdx.x; it < nu * 8; it += kThreads) {
+        // One pass over the chunk's items, each thread on its own item (at the
+        // 8B shape every item has a thread), so that no thread takes a key and
+        // a query row one after the other: items [0, nu*8) are the new keys,
+        // the rest the query rows.
+        for (int it = threadIdx.x; it < nu * 8 + nu * M * 8; it += kThreads) {
+            if (it >= nu * 8) {
+                query_item(it - nu * 8, u0);
+                continue;
+            }
+            // New key: rotate, append, capture or stage k0. New value: append.
             const int lu = it >> 3, j = it & 7;
             const int u = u0 + lu;
             // The new key and value do not depend on the slot: load them in the
@@ -184,30 +217,6 @@ __global__ void __launch_bounds__(kThreads, 1) rope_append_route_kernel(PrestepP
                 ks[j] = k0g[j];
                 ks[j + 8] = k0g[j + 8];
             }
-        }
-        // Query rows: rotate into q_out and the staged rows; a sequence with no
-        // valid slot gets a zero query.
-        for (int it = threadIdx.x; it < nu * M * 8; it += kThreads) {
-            const int r = it >> 3, j = it & 7;
-            const int u = u0 + r / M;
-            const size_t row = ((size_t)u0 * M + r) * kHeadDim;
-            // plain loads: q_out may be q_in (rotated in place)
-            const uint4 *qi = reinterpret_cast<const uint4 *>(p.q_in + row);
-            const uint4 qlo = qi[j], qhi = qi[j + 8];
-            const int pos = slot_of(p, u / p.Hkv);
-            uint4 *qs = rows + r * 16;
-            uint4 *qd = reinterpret_cast<uint4 *>(p.q_out + row);
-            uint4 lo = zero, hi = zero;
-            if (pos >= 0) {
-                float4 c[2], s[2];
-                load_table8(p.rope_cos, pos, j, c);
-                load_table8(p.rope_sin, pos, j, s);
-                rope8(qlo, qhi, c, s, lo, hi);
-            }
-            qs[j] = lo;
-            qs[j + 8] = hi;
-            qd[j] = lo;
-            qd[j + 8] = hi;
         }
         __syncthreads();
         route_units_warp<M, false>(rows, krows, nu, p.tau, (int)threadIdx.x >> 5, kWarps, [&](int lu, bool sink) {
