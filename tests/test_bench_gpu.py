@@ -45,3 +45,26 @@ def test_isolated_step_graph_events_outlive_the_call():
     g.replay()
     torch.cuda.synchronize()
     assert all(e[0].elapsed_time(e[2]) > 0 for e in g.sr_events)
+
+
+def test_append_back_to_back_small():
+    """The back-to-back append timing: every input set's visits append at its
+    last slots, the lengths end at the full context after the timed replay, the
+    routing keeps the planted groups, and no device error is raised."""
+    xs = [inputs.make("tiny_4k", seed=s, device="cuda", max_ctx=512) for s in (5, 6, 7)]
+    x = xs[0]
+    dec = native.Decoder(x.batch, x.n_q_heads, x.n_kv_heads, x.max_seq_len)
+    steps = 7
+    visits = -(-steps // len(xs))
+    seqs = [bench.AppendSequence(native, inputs, xi, visits) for xi in xs]
+    ms = bench.time_append_back_to_back(native, dec, xs, seqs, x.tau, steps, 3)
+    gc.collect()
+    assert ms > 0
+    assert dec.workspace.device_error() == 0
+    for i, (xi, a) in enumerate(zip(xs, seqs)):
+        done = len(range(i, steps, len(xs)))  # this set's visits in one replay
+        assert torch.equal(a.seq_lens, a.seq_saved + done)
+        assert torch.equal(a.seq_saved, xi.seq_lens - visits)
+    # the last step ran on set (steps - 1) % 3: its planted sinks are groups 0-3
+    assert int(dec.active_list[0]) == 4
+    assert dec.route_mask.cpu().tolist() == [1, 1, 1, 1, 0, 0, 0, 0]
