@@ -216,6 +216,24 @@ sr_status sr_decode_attention_lse(const sr_dims *dims, const void *q, const void
                                   size_t workspace_bytes, void *stream);
 
 /*
+ * sr_position0_weight -- the full-attention weight of position 0 for every query
+ * head, from the log-sum-exp that sr_decode_attention_lse returns:
+ *     p0[b, h] = exp(<q[b, h], k_cache[b, g, 0]> / sqrt(d) - lse[b, h]),  g = h / M
+ * (fp32 dot product of the bf16 rows). The pith.science review of arXiv
+ * 2604.16883 (Figure 10 caption) defines the routing proxy's reference "oracle
+ * sink event" from these weights. Heads whose lse is NaN (sinks) get NaN.
+ *
+ *   q        bf16 [B, Hq, d], 16-byte aligned: the query the lse was computed for
+ *   k_cache  bf16 [B, Hkv, Lmax, d], 16-byte aligned: position 0 of every unit is read
+ *   lse      fp32 [B, Hq], device, 4-byte aligned
+ *   p0       out fp32 [B, Hq], device, 4-byte aligned
+ * One launch (one warp per head), asynchronous on `stream`, no workspace.
+ * Errors: SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_CUDA.
+ */
+sr_status sr_position0_weight(const sr_dims *dims, const void *q, const void *k_cache, const float *lse,
+                              float *p0, void *stream);
+
+/*
  * sr_route_decode_attention -- sr_route followed by sr_decode_attention in ONE
  * kernel launch: every CTA of the decode kernel routes all units itself (the
  * same fp32 arithmetic as sr_route, so the decisions are identical) and builds

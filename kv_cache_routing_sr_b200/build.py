@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libsinkrouter.so")
 SOURCES = ["sr_abi.cu", "sr_route.cu", "sr_prestep.cu", "sr_decode.cu", "sr_combine.cu", "sr_static_scratch.cu",
-           "sr_selftest.cu"]
+           "sr_selftest.cu", "sr_position0.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

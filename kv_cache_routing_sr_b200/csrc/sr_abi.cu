@@ -258,6 +258,20 @@ sr_status sr_combine_partials(const sr_dims *dims, int32_t n_parts, const float 
     return e == cudaSuccess ? SR_OK : cuda_fail(e);
 }
 
+sr_status sr_position0_weight(const sr_dims *dims, const void *q, const void *k_cache, const float *lse, float *p0,
+                              void *stream)
+{
+    const sr_status st = check_dims(dims);
+    if (st != SR_OK)
+        return st;
+    if (!q || !k_cache || !lse || !p0 || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(lse, 4) ||
+        !aligned(p0, 4))
+        return SR_ERR_INVALID_ARG;
+    const cudaError_t e = sr::launch_position0(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->max_seq_len, q,
+                                               k_cache, lse, p0, as_stream(stream));
+    return e == cudaSuccess ? SR_OK : cuda_fail(e);
+}
+
 sr_status sr_selftest_bounded_wait(int32_t limit_us, int32_t *status, uint64_t *waited_ns, void *stream)
 {
     if (limit_us < 1 || limit_us > 2000000 || !status || !aligned(status, 4) || !waited_ns || !aligned(waited_ns, 8))

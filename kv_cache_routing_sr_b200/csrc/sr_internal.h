@@ -91,6 +91,9 @@ cudaError_t launch_rope_append_route(const PrestepArgs &a, cudaStream_t stream);
 cudaError_t launch_bounded_wait_selftest(int32_t limit_us, int32_t *status, unsigned long long *waited_ns,
                                          cudaStream_t stream);
 // Log-sum-exp combination of n_parts partial outputs (sr_combine_partials).
+// p0[b, h] = exp(<q[b, h], K[b, g, 0]> / sqrt(d) - lse[b, h]) (sr_position0_weight)
+cudaError_t launch_position0(int B, int Hq, int Hkv, int Lmax, const void *q, const void *k_cache, const float *lse,
+                             float *p0, cudaStream_t stream);
 cudaError_t launch_combine(int n_heads, int n_parts, const float *o_parts, const float *lse_parts, int64_t part_stride,
                            void *out, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);

@@ -43,7 +43,7 @@ EXPORTS = ["sr_route", "sr_decode_workspace_bytes", "sr_workspace_init", "sr_dec
            "sr_status_string", "sr_get_device_error", "sr_clear_device_error", "sr_decode_grid_size",
            "sr_last_cuda_error", "sr_decode_attention_static_scratch", "sr_route_decode_attention",
            "sr_decode_attention_lse", "sr_rope_append_route", "sr_decode_attention_partial",
-           "sr_combine_partials", "sr_selftest_bounded_wait"]
+           "sr_combine_partials", "sr_selftest_bounded_wait", "sr_position0_weight"]
 
 
 def load(path: str | None = None):
@@ -94,6 +94,8 @@ def load(path: str | None = None):
     lib.sr_route_decode_attention.restype = ctypes.c_int
     lib.sr_decode_attention_lse.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, u64, vp]
     lib.sr_decode_attention_lse.restype = ctypes.c_int
+    lib.sr_position0_weight.argtypes = [dp, vp, vp, vp, vp, vp]
+    lib.sr_position0_weight.restype = ctypes.c_int
     lib.sr_rope_append_route.argtypes = [dp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                          vp, vp, vp]
     lib.sr_rope_append_route.restype = ctypes.c_int
@@ -224,6 +226,22 @@ def decode_attention(q, k_cache, v_cache, k0, v0, seq_lens, active_list, out=Non
         _check("sr_decode_attention_lse",
                load().sr_decode_attention_lse(*common, _dev(lse, "lse", torch.float32), *tail))
     return out
+
+
+@_on_tensor_device
+def position0_weight(q, k_cache, lse, p0=None, stream=None):
+    """sr_position0_weight: p0 fp32 [B, Hq], the full-attention weight of
+    position 0 of every head, from the lse of sr_decode_attention_lse."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if p0 is None:
+        p0 = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    dims = dims_of(B, Hq, Hkv, Lmax, d)
+    _check("sr_position0_weight",
+           load().sr_position0_weight(ctypes.byref(dims), _dev(q, "q", torch.bfloat16),
+                                      _dev(k_cache, "k_cache", torch.bfloat16), _dev(lse, "lse", torch.float32),
+                                      _dev(p0, "p0", torch.float32), _stream(stream)))
+    return p0
 
 
 @_on_tensor_device

@@ -10,7 +10,7 @@ functions of the threshold (operating point 0.55). Here, on synthetic inputs:
   full-attention weight of position 0, p0, is at least `cutoff` (the pages do
   not define the event exactly; this is the reading taken);
 * p0 comes from the decode kernel run with routing disabled, through its
-  log-sum-exp output: p0 = exp(<q_h, K_0> / sqrt(d) - lse_h);
+  log-sum-exp output and sr_position0_weight: p0 = exp(<q_h, K_0> / sqrt(d) - lse_h);
 * the proxy decision at threshold tau is sr_route's mask (min over the group's
   heads of the cosine with k0, >= tau).
 
@@ -47,15 +47,12 @@ def pr_curve(scores_by_tau: dict, event: torch.Tensor) -> list:
 def full_attention_p0(x: _inputs.DecodeInputs) -> torch.Tensor:
     """p0 [B, Hq] of dense attention (routing disabled) via the kernel's lse."""
     B, Hq, Hkv = x.batch, x.n_q_heads, x.n_kv_heads
-    M = Hq // Hkv
     dec = native.Decoder(B, Hq, Hkv, x.max_seq_len, device=x.q.device)
     native.route(x.q, x.k0, math.inf, dec.route_mask, dec.active_list)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=x.q.device)
     native.decode_attention(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, dec.active_list, dec.out,
                             workspace=dec.workspace, lse=lse)
-    k_first = x.k_cache[:, :, 0].float().repeat_interleave(M, dim=1)  # [B, Hq, d]
-    logit0 = (x.q.float() * k_first).sum(-1) / math.sqrt(x.q.shape[-1])
-    return torch.exp(logit0 - lse)
+    return native.position0_weight(x.q, x.k_cache, lse)
 
 
 def evaluate(x: _inputs.DecodeInputs, taus, cutoff: float = 0.5) -> dict:

@@ -528,3 +528,22 @@ def test_concurrent_host_threads_on_separate_streams():
         assert len(results[i]) == 30
         for out in results[i]:
             assert torch.equal(out.cpu().view(torch.int16), refs[i].cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (64, 8)])
+def test_position0_weight_matches_its_definition(Hq, Hkv):
+    """sr_position0_weight against exp(<q, K[., g, 0]> / sqrt(d) - lse) in fp64,
+    for given lse values (NaN ones propagate), at M = 1, 4 and 8."""
+    g = torch.Generator(device=DEV).manual_seed(Hq * 7 + Hkv)
+    B, L = 3, 40
+    q = torch.randn((B, Hq, 128), generator=g, device=DEV).to(torch.bfloat16)
+    kc = torch.randn((B, Hkv, L, 128), generator=g, device=DEV).to(torch.bfloat16)
+    lse = (torch.rand((B, Hq), generator=g, device=DEV) * 4.0 + 1.0).float()
+    lse[0, 1] = float("nan")
+    p0 = native.position0_weight(q, kc, lse).cpu().double()
+    M = Hq // Hkv
+    k0 = kc[:, :, 0].cpu().double().repeat_interleave(M, dim=1)
+    ref = torch.exp((q.cpu().double() * k0).sum(-1) / math.sqrt(128) - lse.cpu().double())
+    assert torch.isnan(p0[0, 1]) and torch.isnan(ref[0, 1])
+    ok = ~torch.isnan(ref)
+    assert ((p0[ok] - ref[ok]).abs() / ref[ok]).max().item() < 1e-5
