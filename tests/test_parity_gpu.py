@@ -547,3 +547,25 @@ def test_position0_weight_matches_its_definition(Hq, Hkv):
     assert torch.isnan(p0[0, 1]) and torch.isnan(ref[0, 1])
     ok = ~torch.isnan(ref)
     assert ((p0[ok] - ref[ok]).abs() / ref[ok]).max().item() < 1e-5
+
+
+def test_two_million_positions_every_unit():
+    """Contexts four times the longest workload (2^21 positions, one sequence
+    77 short of it): 64-bit offsets, long shares and the tail tile, on every
+    unit at M = 8 with routing off, against the oracle element by element."""
+    import types
+    g = torch.Generator(device=DEV).manual_seed(2021)
+    B, Hkv, M, L = 2, 1, 8, 1 << 21
+    q = (2.0 * torch.randn((B, Hkv * M, 128), generator=g, device=DEV)).to(torch.bfloat16)
+    kc = torch.randn((B, Hkv, L, 128), generator=g, device=DEV).to(torch.bfloat16)
+    vc = torch.randn((B, Hkv, L, 128), generator=g, device=DEV).to(torch.bfloat16)
+    sl = torch.tensor([L, L - 77], dtype=torch.int32, device=DEV)
+    x = types.SimpleNamespace(q=q, k_cache=kc, v_cache=vc, k0=kc[:, :, 0].contiguous(), v0=vc[:, :, 0].contiguous(),
+                              seq_lens=sl, batch=B, n_q_heads=Hkv * M, n_kv_heads=Hkv, max_seq_len=L)
+    dec = native.Decoder(B, Hkv * M, Hkv, L)
+    out = dec.step(x.q, x.k_cache, x.v_cache, x.k0, x.v0, x.seq_lens, float("inf"))
+    torch.cuda.synchronize()
+    assert dec.workspace.device_error() == 0
+    mask = dec.route_mask.cpu()
+    assert int(mask.sum()) == 0
+    H.check_against_oracle(x, out.cpu(), mask, what="2M positions")
