@@ -6,14 +6,19 @@ sr_decode_attention, through the C ABI) on synthetic inputs shaped like the
 Llama-3.1-8B 128K-context decode layer: batch 1, 32 query / 8 KV heads,
 head_dim 128, bf16 cache, 4 of 8 KV groups planted sinks, tau 0.6.
 
+Timing: K layer-steps back to back in one CUDA graph, rotating over input sets
+that together exceed L2, one event pair around all of them; the graph is
+replayed once untimed, then once timed.
+
 Prints one JSON line (rank 0): µs per layer-step (lower is better), effective
 HBM GB/s over the bytes the step must move, the roofline of the decode kernel
-against the measured HBM copy bandwidth, the same kernel with routing disabled
-(tau = +inf), the fused single launch, the append step (RoPE + KV append +
-routing, then the scan), the 512K sink-fraction sweep and the other workloads
-(one GPU), the fp64 CPU oracle on this host's cores, end-to-end figures with
-host buffers (every input each step; and the serving view, only the new token's
-projections), and the SM clocks seen during the timed region.
+against the HBM copy bandwidth (measured, else the fallback), the same kernel
+with routing disabled (tau = +inf), the fused single launch, the per-step
+protocol (flush, events) for comparison, the append step (RoPE + KV append +
+routing, then the scan), the 512K sink-fraction sweep, short contexts and the
+other workloads (one GPU), the fp64 CPU oracle on this host's cores, end-to-end
+figures with host buffers (every input each step; and the serving view, only
+the new token's projections), and the SM clocks seen during the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --multilayer        # per-token latency of a gated 32-layer graph
