@@ -81,7 +81,12 @@ constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 constexpr float kScaleLog2 = 0.12751743082459868f; // log2(e) / sqrt(128)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMergeThreads = 32 * kCWarps;
-constexpr int kMergeBatch = 16; // partials in flight per thread in the final merge
+// Partials in flight per thread in the final merge (at most 32: lane k of a
+// warp loads the (m, l) of the batch's k-th partial). Each batch costs one
+// round trip for lines other SMs have just written (~0.9 us); 25 covers the 74
+// partials of a unit at 512K with 2 of 8 units active in 3 batches, and the 37
+// at 128K with 4 active in 2.
+constexpr int kMergeBatch = 25;
 // Row stride (floats) of the split-end scratch that holds each warp's O per
 // head: 4 floats of padding put the lanes that store the same row of
 // different head pairs in different banks.
@@ -1092,36 +1097,40 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     const int head = col >> 5, d4 = (col & 31) * 4;
                     float m = -INFINITY, l = 0.f;
                     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    // All lanes of a warp share the head and the partial group:
+                    // lane k loads the (m, l) of the batch's k-th partial and
+                    // the weights reach the other lanes by shuffles, so only
+                    // the O values take registers in every lane.
                     for (int j0 = grp; j0 < h.nseg; j0 += sgrp * kMergeBatch) {
-                        float2 x[kMergeBatch];
+                        const int jl = j0 + lane * sgrp;
+                        float2 xl = make_float2(-INFINITY, 0.f);
+                        if (lane < kMergeBatch && jl < h.nseg)
+                            xl = __ldcg(p.part_ml + (size_t)(h.slot_first + jl) * M + head);
                         float4 y[kMergeBatch];
 #pragma unroll
                         for (int k = 0; k < kMergeBatch; ++k) {
                             const int j = j0 + k * sgrp;
-                            if (j < h.nseg) {
-                                const size_t sl = (size_t)(h.slot_first + j) * M + head;
-                                x[k] = __ldcg(p.part_ml + sl);
-                                y[k] = __ldcg(reinterpret_cast<const float4 *>(p.part_o + sl * kHeadDim + d4));
-                            } else {
-                                x[k] = make_float2(-INFINITY, 0.f);
-                                y[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            }
+                            y[k] = (j < h.nseg) ? __ldcg(reinterpret_cast<const float4 *>(
+                                                      p.part_o + ((size_t)(h.slot_first + j) * M + head) * kHeadDim + d4))
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
                         }
-                        // One rescale per batch: the batch maximum first,
-                        // then independent weights (empty splits weigh 0).
-                        float mb = -INFINITY;
+                        float mb = xl.x;
 #pragma unroll
-                        for (int k = 0; k < kMergeBatch; ++k)
-                            mb = fmaxf(mb, x[k].x);
+                        for (int off = 16; off > 0; off >>= 1)
+                            mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
                         const float mn = fmaxf(m, mb);
                         if (mn != -INFINITY) {
                             const float a = exp2f(m - mn);
-                            l *= a;
+                            const float cw = (xl.x == -INFINITY) ? 0.f : exp2f(xl.x - mn);
+                            float ls = xl.y * cw;
+#pragma unroll
+                            for (int off = 16; off > 0; off >>= 1)
+                                ls += __shfl_xor_sync(kFull, ls, off);
+                            l = l * a + ls;
                             acc.x *= a, acc.y *= a, acc.z *= a, acc.w *= a;
 #pragma unroll
                             for (int k = 0; k < kMergeBatch; ++k) {
-                                const float c = exp2f(x[k].x - mn);
-                                l += x[k].y * c;
+                                const float c = __shfl_sync(kFull, cw, k);
                                 acc.x += y[k].x * c;
                                 acc.y += y[k].y * c;
                                 acc.z += y[k].z * c;
