@@ -443,7 +443,7 @@ def test_proxy_quality_analysis_runs_and_matches_oracle_event():
     assert torch.equal((p0 >= 0.5)[~near], ev_ref[~near])
 
 
-@pytest.mark.parametrize("M,ns,L", [(4, 70, 9000), (8, 40, 6000), (1, 140, 20000), (2, 7, 3000)])
+@pytest.mark.parametrize("M,ns,L", [(4, 70, 9000), (8, 40, 6000), (1, 140, 20000), (2, 7, 3000), (2, 66, 9000)])
 def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
     """With forced splits a unit's partials depend only on n_splits and its
     length, and the last-CTA merge takes them in a fixed order, so unit 0's
@@ -452,8 +452,8 @@ def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
     further work) against unit 0 among many active units (more splits than
     CTAs: CTA j's split j is never its last), and the first sequence as a
     launch of its own, whose 8 units take the prologue's register path.
-    ns = 70 at M = 4, 40 at M = 8 and 140 at M = 1 take several batches of the
-    merge."""
+    ns = 70 at M = 4, 40 at M = 8, 140 at M = 1 and 66 at M = 2 take several
+    batches of the merge (at M < 4 in several partial groups)."""
     G = native.grid_size()
     Hkv = 8
     B = max(1, -(-(G + ns) // (ns * Hkv)) + 1)  # B*Hkv*ns > G + ns
@@ -481,6 +481,10 @@ def test_unit_result_independent_of_the_rest_of_the_launch(M, ns, L):
         assert ws.device_error() == 0
         runs[name] = (out[0, :M].cpu(), lse[0, :M].cpu())
     a = runs["alone"]
+    # and unit 0 itself against the oracle (one-unit sub-problem, routed active)
+    ref, _ = oracle.decode(q[:1, :M].cpu(), kc[:1, :1].cpu(), vc[:1, :1].cpu(), v0[:1, :1].cpu(), sl[:1].cpu(),
+                           torch.zeros(1, dtype=torch.uint8))
+    H.assert_active_close(a[0].unsqueeze(0), ref, f"unit 0, M={M}, {ns} forced splits")
     for other in ("among_many", "one_sequence"):
         b = runs[other]
         assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)), f"unit 0 differs ({other})"
