@@ -528,6 +528,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 
     const int G = gridDim.x;
     long long chunk = 1, r0 = 0, r1 = 0;
+    // The producer lane issued the copies of its first tile before finishing
+    // the plan; its first emit only writes the header and arrives.
+    bool early = false;
     if (p.n_splits == 0 && P > 0) {
         chunk = div_nonneg(P + G - 1, G);
         chunk = (chunk + C::BN - 1) / C::BN * C::BN;
@@ -551,6 +554,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 i0 = gt ? i : INT_MAX;
             }
             const int fu = (i0 < n) ? __shfl_sync(kFull, lane_unit, i0 < 32 ? i0 : 0) : -1;
+            const int lb = lane_unit / p.Hkv;
+            const int lane_qrow = lb * p.Hq + (lane_unit - lb * p.Hkv) * M;
+            const int fq = __shfl_sync(kFull, lane_qrow, i0 < 32 ? i0 : 0);
+            if (lane == 0 && p.n_splits == 0 && i0 < n) {
+                // The first tile of this CTA's first split (unit fu from
+                // position r0 - s0, with the group's q rows) into stage 0 now:
+                // its full barrier expects the bytes but cannot complete
+                // before the header is written and the producer arrives.
+                const uint32_t sb = smem_u32(smem);
+                const uint64_t pol0 = l2_policy_evict_first();
+                mbar_expect_tx(full0, (uint32_t)C::STAGE + (uint32_t)(M * kHeadDim * 2));
+                const int pos0 = (int)(r0 - s0);
+                tma_load_3d(sb, &tmK, full0, 0, pos0, fu, pol0);
+                tma_load_3d(sb + C::HALF, &tmK, full0, 64, pos0, fu, pol0);
+                tma_load_3d(sb + 2 * C::HALF, &tmV, full0, 0, pos0, fu, pol0);
+                tma_load_3d(sb + 3 * C::HALF, &tmV, full0, 64, pos0, fu, pol0);
+                const uint8_t *qsrc = reinterpret_cast<const uint8_t *>(p.q + (size_t)fq * kHeadDim);
+                for (int hq = 0; hq < M; ++hq)
+                    bulk_load(smem_u32(smem + C::OFF_Q + hq * kQRowBytes), qsrc + hq * kHeadDim * 2, kHeadDim * 2,
+                              full0);
+                SR_STAMP(tl_decode, 4);
+                early = true;
+            }
             if (lane == 0) {
                 misc->i0 = i0;
                 misc->s0 = s0;
@@ -561,8 +587,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 ri.start = lane_incl - lane_len;
                 ri.unit = lane_unit;
                 ri.len = lane_len;
-                const int b = lane_unit / p.Hkv;
-                ri.qrow = b * p.Hq + (lane_unit - b * p.Hkv) * M;
+                ri.qrow = lane_qrow;
                 ri.cf = (p.n_splits == 0) ? (int)div_nonneg(ri.start, chunk) : 0;
                 ri.cl = (p.n_splits == 0) ? (int)div_nonneg(ri.start + lane_len - 1, chunk) : 0;
                 ri.pad = 0;
@@ -614,6 +639,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 #pragma unroll
         for (int s = 0; s < STAGES; ++s)
             issued_parity[s] = -1;
+        if (early)
+            issued_parity[0] = 0; // the first tile's copies are in flight
         bool ok = true;
 
         auto emit = [&](const TileHdr &h, const void *qsrc, uint32_t qbytes) -> bool {
@@ -630,6 +657,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 #endif
             hdr[stage] = h;
             const uint32_t fb = full0 + 8 * stage;
+            if (early) {
+                // this tile's copies were issued in the prologue (same unit,
+                // position and q rows): publish the header and arrive
+                early = false;
+                mbar_arrive(fb);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    ph ^= 1;
+                }
+                return true;
+            }
             const uint32_t bytes = (h.nvalid > 0 ? (uint32_t)C::STAGE : 0u) + qbytes;
             if (bytes) {
                 mbar_arrive_expect_tx(fb, bytes);
@@ -771,6 +809,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         }
         if (!ok) {
             atomicOr(p.err, SR_DEVERR_TIMEOUT);
+            if (early) // its phase completes only once the producer has arrived
+                mbar_arrive(full0);
             // Let every copy still in flight land before this CTA can exit.
             volatile int never = 0;
             for (int s = 0; s < STAGES; ++s)
